@@ -1,0 +1,280 @@
+"""Python binding of libmuon (include/muon.h): the Muon optimizer step and
+batched Newton-Schulz orthogonalisation on NVIDIA B200.
+
+This module only marshals arguments: it turns torch tensors into device
+pointers, groups, hyper-parameter structs and the current CUDA stream, and calls
+the C ABI through ctypes.  Every step of the computation runs in the library's
+CUDA kernels.  There is no fallback: if ``libmuon.so`` is missing or no CUDA
+device is present, the calls raise.
+
+Build the library with ``python -m newton_schulz_matrix_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+import torch
+
+__all__ = [
+    "BF16", "FP16", "FP32", "STANDARD", "GRAM", "GRAM_STABILIZED", "QUINTIC", "CUBIC",
+    "MuonError", "load_library", "library_path", "muon_step", "muon_ns_batched",
+    "muon_workspace_size", "muon_workspace_min", "muon_ns_workspace_size", "muon_ns_flops",
+    "muon_status_string", "EXPORTED_SYMBOLS",
+]
+
+BF16, FP16, FP32 = 0, 1, 2
+STANDARD, GRAM, GRAM_STABILIZED = 0, 1, 2
+_MODE_NAMES = {"standard": STANDARD, "gram": GRAM, "gram_stabilized": GRAM_STABILIZED}
+_DT_NAMES = {"bf16": BF16, "fp16": FP16, "fp32": FP32}
+QUINTIC = (3.4445, -4.7750, 2.0315)
+CUBIC = (1.5, -0.5, 0.0)
+EXPORTED_SYMBOLS = (
+    "muon_workspace_size", "muon_workspace_min", "muon_step", "muon_ns_workspace_size",
+    "muon_ns_batched", "muon_ns_flops", "muon_status_string",
+)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+
+class MuonError(RuntimeError):
+    pass
+
+
+class _NSParams(ctypes.Structure):
+    _fields_ = [("iters", ctypes.c_int), ("coeffs", ctypes.POINTER(ctypes.c_float)), ("mode", ctypes.c_int),
+                ("restart_after", ctypes.c_int), ("eps", ctypes.c_float), ("compute_dtype", ctypes.c_int),
+                ("gram_dtype", ctypes.c_int)]
+
+
+class _Group(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("count", ctypes.c_int),
+                ("w_dtype", ctypes.c_int), ("g_dtype", ctypes.c_int),
+                ("W", ctypes.POINTER(ctypes.c_void_p)), ("G", ctypes.POINTER(ctypes.c_void_p)),
+                ("M", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class _HParams(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("momentum", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("scale_coef", ctypes.c_float), ("nesterov", ctypes.c_int), ("ns", _NSParams)]
+
+
+def library_path() -> str:
+    return os.environ.get("MUON_LIBRARY", os.path.join(_HERE, "libmuon.so"))
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libmuon.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = library_path()
+    if not os.path.exists(path):
+        raise MuonError(f"{path} is missing: build it with `python -m newton_schulz_matrix_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    lib.muon_workspace_size.argtypes = [ctypes.POINTER(_Group), ctypes.c_int, ctypes.POINTER(_HParams)]
+    lib.muon_workspace_size.restype = ctypes.c_size_t
+    lib.muon_workspace_min.argtypes = [ctypes.POINTER(_Group), ctypes.c_int, ctypes.POINTER(_HParams)]
+    lib.muon_workspace_min.restype = ctypes.c_size_t
+    lib.muon_step.argtypes = [ctypes.POINTER(_Group), ctypes.c_int, ctypes.POINTER(_HParams), P, ctypes.c_size_t,
+                              P, P]
+    lib.muon_step.restype = ctypes.c_int
+    lib.muon_ns_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(_NSParams)]
+    lib.muon_ns_workspace_size.restype = ctypes.c_size_t
+    lib.muon_ns_batched.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.POINTER(_NSParams), P, ctypes.c_size_t, P, P]
+    lib.muon_ns_batched.restype = ctypes.c_int
+    lib.muon_ns_flops.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_NSParams)]
+    lib.muon_ns_flops.restype = ctypes.c_double
+    lib.muon_status_string.argtypes = [ctypes.c_int]
+    lib.muon_status_string.restype = ctypes.c_char_p
+    _LIB = lib
+    return lib
+
+
+# ---------------------------------------------------------------------------
+# argument marshalling
+# ---------------------------------------------------------------------------
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float16:
+        return FP16
+    if t == torch.float32:
+        return FP32
+    raise MuonError(f"unsupported dtype {t}")
+
+
+def _code(v, names) -> int:
+    return names[v] if isinstance(v, str) else int(v)
+
+
+def _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype):
+    flat = [float(x) for abc in coeffs for x in abc]
+    arr = (ctypes.c_float * len(flat))(*flat)
+    p = _NSParams(len(flat) // 3, ctypes.cast(arr, ctypes.POINTER(ctypes.c_float)), _code(mode, _MODE_NAMES),
+                  int(restart_after), float(eps), _code(compute_dtype, _DT_NAMES), _code(gram_dtype, _DT_NAMES))
+    return p, arr
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check_cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise MuonError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise MuonError(f"{name} must be contiguous (row-major)")
+    if t.dim() != 2:
+        raise MuonError(f"{name} must be 2-D")
+
+
+def _raise(rc: int, what: str):
+    if rc != 0:
+        raise MuonError(f"{what} failed: {rc} ({muon_status_string(rc)})")
+
+
+def _build_groups(params, grads, moms):
+    """Group tensors by (shape, W dtype, G dtype) in first-appearance order."""
+    keys = []
+    index = {}
+    for i, (w, g, m) in enumerate(zip(params, grads, moms)):
+        _check_cuda(w, "param"); _check_cuda(g, "grad"); _check_cuda(m, "momentum")
+        if w.shape != g.shape or w.shape != m.shape:
+            raise MuonError("param, grad and momentum shapes differ")
+        if m.dtype != torch.float32:
+            raise MuonError("momentum buffers must be float32")
+        k = (tuple(w.shape), _dtype_code(w.dtype), _dtype_code(g.dtype))
+        if k not in index:
+            index[k] = len(keys)
+            keys.append((k, []))
+        keys[index[k]][1].append(i)
+    groups = (_Group * len(keys))()
+    keep = []
+    order = []
+    for gi, ((shape, wdt, gdt), idx) in enumerate(keys):
+        n = len(idx)
+        W = (ctypes.c_void_p * n)(*[params[i].data_ptr() for i in idx])
+        G = (ctypes.c_void_p * n)(*[grads[i].data_ptr() for i in idx])
+        M = (ctypes.c_void_p * n)(*[moms[i].data_ptr() for i in idx])
+        keep += [W, G, M]
+        groups[gi] = _Group(shape[0], shape[1], n, wdt, gdt, W, G, M)
+        order += idx
+    return groups, len(keys), keep, order
+
+
+def _hparams(lr, momentum, weight_decay, scale_coef, nesterov, ns):
+    return _HParams(float(lr), float(momentum), float(weight_decay), float(scale_coef), int(bool(nesterov)), ns)
+
+
+# ---------------------------------------------------------------------------
+# public API (same names as the C ABI)
+# ---------------------------------------------------------------------------
+def muon_status_string(code: int) -> str:
+    return load_library().muon_status_string(int(code)).decode()
+
+
+def muon_ns_flops(rows: int, cols: int, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2) -> float:
+    ns, _arr = _ns_params(coeffs, mode, restart_after, 1e-7, BF16, FP16)
+    return load_library().muon_ns_flops(rows, cols, ctypes.byref(ns))
+
+
+def _step_args(params, grads, moms, lr, momentum, nesterov, weight_decay, scale_coef, eps, coeffs, mode,
+               restart_after, compute_dtype, gram_dtype):
+    if not (len(params) == len(grads) == len(moms)) or len(params) == 0:
+        raise MuonError("params, grads and moms must be non-empty lists of equal length")
+    groups, ng, keep, order = _build_groups(params, grads, moms)
+    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+    hp = _hparams(lr, momentum, weight_decay, scale_coef, nesterov, ns)
+    return groups, ng, hp, (keep, arr), order
+
+
+_STEP_DEFAULTS = dict(lr=0.02, momentum=0.95, nesterov=True, weight_decay=0.1, scale_coef=0.2, eps=1e-7,
+                      coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2, compute_dtype="bf16",
+                      gram_dtype="fp16")
+
+
+def muon_workspace_size(params, grads, moms, **hp) -> int:
+    a = dict(_STEP_DEFAULTS, **hp)
+    groups, ng, h, _keep, _ = _step_args(params, grads, moms, **a)
+    return int(load_library().muon_workspace_size(groups, ng, ctypes.byref(h)))
+
+
+def muon_workspace_min(params, grads, moms, **hp) -> int:
+    a = dict(_STEP_DEFAULTS, **hp)
+    groups, ng, h, _keep, _ = _step_args(params, grads, moms, **a)
+    return int(load_library().muon_workspace_min(groups, ng, ctypes.byref(h)))
+
+
+def muon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor], moms: Sequence[torch.Tensor], *,
+              workspace: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None,
+              **hp) -> torch.Tensor | None:
+    """One Muon step, in place on ``params`` and ``moms``.
+
+    Keyword hyper-parameters (defaults: lr 0.02, momentum 0.95, nesterov True,
+    weight_decay 0.1, scale_coef 0.2, eps 1e-7, five quintic iterations,
+    mode "standard", restart_after 2, compute_dtype "bf16", gram_dtype "fp16").
+    ``workspace`` is a CUDA uint8 tensor (allocated when None); ``status``, if
+    given, is an int32 CUDA tensor with one word per parameter (in the order of
+    ``params``) and receives the MUON_STATUS_* bits.
+    """
+    lib = load_library()
+    a = dict(_STEP_DEFAULTS, **hp)
+    groups, ng, h, keep, order = _step_args(params, grads, moms, **a)
+    need = int(lib.muon_workspace_size(groups, ng, ctypes.byref(h)))
+    if need == 0:
+        raise MuonError("invalid arguments (workspace query returned 0)")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=params[0].device)
+    st_grouped = None
+    if status is not None:
+        st_grouped = torch.empty(len(order), dtype=torch.int32, device=params[0].device)
+    rc = lib.muon_step(groups, ng, ctypes.byref(h), ctypes.c_void_p(workspace.data_ptr()),
+                       ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                       ctypes.c_void_p(st_grouped.data_ptr() if st_grouped is not None else 0),
+                       ctypes.c_void_p(_stream_handle(stream)))
+    _raise(rc, "muon_step")
+    if status is not None:
+        status[torch.tensor(order, device=status.device)] = st_grouped
+    return status
+
+
+def muon_ns_workspace_size(count: int, rows: int, cols: int, coeffs=(QUINTIC,) * 5, mode="standard",
+                           restart_after=2, eps=1e-7, compute_dtype="bf16", gram_dtype="fp16") -> int:
+    ns, _arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+    return int(load_library().muon_ns_workspace_size(count, rows, cols, ctypes.byref(ns)))
+
+
+def muon_ns_batched(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2,
+                    eps=1e-7, compute_dtype=None, gram_dtype="fp16", workspace: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None, stream=None) -> None:
+    """Orthogonalise same-shape matrices in place (result has each input's shape)."""
+    lib = load_library()
+    if len(X) == 0:
+        return
+    for t in X:
+        _check_cuda(t, "X")
+        if t.shape != X[0].shape or t.dtype != X[0].dtype:
+            raise MuonError("all matrices must share shape and dtype")
+    rows, cols = X[0].shape
+    dt = _dtype_code(X[0].dtype)
+    if compute_dtype is None:
+        compute_dtype = "fp32" if dt == FP32 else "bf16"
+    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+    need = int(lib.muon_ns_workspace_size(len(X), rows, cols, ctypes.byref(ns)))
+    if need == 0:
+        raise MuonError("invalid arguments (workspace query returned 0)")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X[0].device)
+    ptrs = (ctypes.c_void_p * len(X))(*[t.data_ptr() for t in X])
+    rc = lib.muon_ns_batched(ptrs, len(X), rows, cols, dt, ctypes.byref(ns), ctypes.c_void_p(workspace.data_ptr()),
+                             ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                             ctypes.c_void_p(status.data_ptr() if status is not None else 0),
+                             ctypes.c_void_p(_stream_handle(stream)))
+    _raise(rc, "muon_ns_batched")

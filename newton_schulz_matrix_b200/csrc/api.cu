@@ -1,0 +1,532 @@
+// C ABI of libmuon (include/muon.h): argument checks, the shape planner that
+// merges groups by oriented shape and cuts them into workspace-sized chunks,
+// the workspace layout, and the launch sequence of one Muon step:
+//
+//   pack (momentum, Nesterov, orientation, sums of squares)  -> norm
+//   -> Newton-Schulz chain of tensor-core products            -> unpack (update)
+//
+// The iteration order follows the "Gram Newton-Schulz" write-up (standard
+// form: A = X X^T, B = b A + c A^2, X = a X + B X; Gram form: iterate on
+// R = X X^T, accumulate Q_acc = Q_k ... Q_1, restart once in the stabilised
+// variant) and the optimizer step of "Moonlight 16B Guide" (box steps 1-4).
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+#include <vector>
+
+#include "../../include/muon.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace muon;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline int round8(int v) { return (v + 7) / 8 * 8; }
+
+struct Seg {          // `count` matrices of one caller group, starting at index `first`
+  int group, first, count;
+};
+
+struct Batch {        // matrices that orient to the same n x m
+  int n, m;
+  std::vector<Seg> segs;
+  int total = 0;
+};
+
+struct Layout {       // per-chunk workspace layout for a batch
+  int n, m, ld_m, ld_n;
+  int x_es, g_es;     // element sizes of X and Gram buffers
+  int n_sq;           // number of n x n buffers
+  int tiles;          // pack tiles per matrix (sums-of-squares partials)
+  size_t per_matrix;  // bytes per matrix (all buffers)
+  size_t fixed;       // bytes independent of the chunk size
+};
+
+bool ns_params_ok(const muon_ns_params* ns) {
+  if (!ns || ns->iters < 1 || ns->iters > 1000 || !ns->coeffs) return false;
+  if (ns->mode < MUON_NS_STANDARD || ns->mode > MUON_NS_GRAM_STABILIZED) return false;
+  if (ns->mode == MUON_NS_GRAM_STABILIZED && (ns->restart_after < 1 || ns->restart_after >= ns->iters)) return false;
+  if (!(ns->eps >= 0.f) || !std::isfinite(ns->eps)) return false;
+  if (ns->compute_dtype < MUON_BF16 || ns->compute_dtype > MUON_FP32) return false;
+  if (ns->mode != MUON_NS_STANDARD && ns->compute_dtype != MUON_FP32 && ns->gram_dtype != MUON_BF16 &&
+      ns->gram_dtype != MUON_FP16)
+    return false;
+  for (int i = 0; i < 3 * ns->iters; ++i)
+    if (!std::isfinite(ns->coeffs[i])) return false;
+  return true;
+}
+
+bool dtype_ok(int d) { return d == MUON_BF16 || d == MUON_FP16 || d == MUON_FP32; }
+
+Layout make_layout(int n, int m, const muon_ns_params* ns) {
+  Layout L{};
+  L.n = n; L.m = m;
+  L.ld_m = round8(m);
+  L.ld_n = round8(n);
+  L.x_es = ns->compute_dtype == MUON_FP32 ? 4 : 2;
+  L.g_es = ns->compute_dtype == MUON_FP32 ? 4 : 2;
+  L.n_sq = ns->mode == MUON_NS_STANDARD ? 2 : 5;
+  L.tiles = pack_tiles(n, m);
+  // buffers: 2 X, n_sq Gram-sized, partials, inv (each 256-byte aligned per chunk)
+  L.per_matrix = 2 * (size_t)n * L.ld_m * L.x_es + (size_t)L.n_sq * n * L.ld_n * L.g_es + (size_t)L.tiles * 4 + 4;
+  L.fixed = kAlign * (2 + L.n_sq + 2 + 1) + kAlign;  // alignment slack + error word
+  return L;
+}
+
+size_t chunk_bytes(const Layout& L, int chunk) { return L.fixed + L.per_matrix * (size_t)chunk; }
+
+struct Bufs {
+  void* X[2];
+  void* S[5];
+  float* partials;
+  float* inv;
+  int* err;
+  long long x_bs, s_bs;
+};
+
+Bufs carve(const Layout& L, int chunk, void* ws) {
+  Bufs B{};
+  char* p = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), kAlign));
+  B.err = reinterpret_cast<int*>(p);
+  p += kAlign;
+  B.x_bs = (long long)L.n * L.ld_m;
+  B.s_bs = (long long)L.n * L.ld_n;
+  for (int i = 0; i < 2; ++i) {
+    B.X[i] = p;
+    p += align_up((size_t)chunk * B.x_bs * L.x_es, kAlign);
+  }
+  for (int i = 0; i < L.n_sq; ++i) {
+    B.S[i] = p;
+    p += align_up((size_t)chunk * B.s_bs * L.g_es, kAlign);
+  }
+  B.partials = reinterpret_cast<float*>(p);
+  p += align_up((size_t)chunk * L.tiles * 4, kAlign);
+  B.inv = reinterpret_cast<float*>(p);
+  return B;
+}
+
+std::vector<Batch> plan_groups(const muon_group* groups, int n_groups) {
+  std::vector<Batch> out;
+  for (int g = 0; g < n_groups; ++g) {
+    const int n = std::min(groups[g].rows, groups[g].cols), m = std::max(groups[g].rows, groups[g].cols);
+    if (groups[g].count == 0) continue;
+    Batch* b = nullptr;
+    for (auto& x : out)
+      if (x.n == n && x.m == m) b = &x;
+    if (!b) {
+      out.push_back(Batch{n, m, {}, 0});
+      b = &out.back();
+    }
+    b->segs.push_back(Seg{g, 0, groups[g].count});
+    b->total += groups[g].count;
+  }
+  return out;
+}
+
+// ------------------------------------------------------------------ products
+struct Ctx {
+  int compute;   // MUON_BF16 / MUON_FP16 / MUON_FP32
+  cudaStream_t s;
+  int* err;
+};
+
+int gemm(const Ctx& c, GemmDesc g) {
+  g.err = c.err;
+  return c.compute == MUON_FP32 ? gemm_simt(g, c.s) : gemm_tc(g, c.s);
+}
+
+GemmDesc desc(int M, int N, int K, int batch) {
+  GemmDesc g{};
+  g.M = M; g.N = N; g.K = K; g.batch = batch;
+  g.c_acc = 1.f;
+  g.b_kmajor = 1;
+  return g;
+}
+
+// Runs the Newton-Schulz chain on `chunk` packed matrices; returns the index of
+// the X buffer that holds the result through *out_x.
+int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, int* out_x) {
+  const int n = L.n, m = L.m, K = ns->iters;
+  const int xdt = c.compute;                                            // X storage
+  const int gdt = c.compute == MUON_FP32 ? MUON_FP32 : ns->gram_dtype;  // Gram storage
+  int rc;
+  if (ns->mode == MUON_NS_STANDARD) {
+    int cur = 0;
+    for (int k = 0; k < K; ++k) {
+      const float a = ns->coeffs[3 * k], bb = ns->coeffs[3 * k + 1], cc = ns->coeffs[3 * k + 2];
+      const bool first = k == 0;
+      // A = f^2 X X^T  (f = 1/(||U||+eps) on the first iteration)
+      GemmDesc g = desc(n, n, m, chunk);
+      g.A = B.X[cur]; g.lda = L.ld_m; g.a_bs = B.x_bs;
+      g.B = B.X[cur]; g.ldb = L.ld_m; g.b_bs = B.x_bs; g.b_kmajor = 1;
+      g.in_dtype = xdt;
+      g.D = B.S[0]; g.ldd = L.ld_n; g.d_bs = B.s_bs; g.d_dtype = xdt;
+      g.scale = B.inv; g.scale_pow = first ? 2 : 0;
+      g.symmetric = 1;
+      if ((rc = gemm(c, g))) return rc;
+      const void* Bm = B.S[0];
+      float coefB = bb;
+      if (cc != 0.f) {
+        // B = c A A + b A   (A symmetric: A A = A A^T)
+        g = desc(n, n, n, chunk);
+        g.A = B.S[0]; g.lda = L.ld_n; g.a_bs = B.s_bs;
+        g.B = B.S[0]; g.ldb = L.ld_n; g.b_bs = B.s_bs; g.b_kmajor = 1;
+        g.in_dtype = xdt;
+        g.D = B.S[1]; g.ldd = L.ld_n; g.d_bs = B.s_bs; g.d_dtype = xdt;
+        g.C = B.S[0]; g.ldc = L.ld_n; g.c_bs = B.s_bs; g.c_dtype = xdt;
+        g.c_acc = cc; g.c_in = bb;
+        g.symmetric = 1;
+        if ((rc = gemm(c, g))) return rc;
+        Bm = B.S[1];
+        coefB = 1.f;
+      }
+      // X' = f (a X + coefB Bm X)
+      g = desc(n, m, n, chunk);
+      g.A = Bm; g.lda = L.ld_n; g.a_bs = B.s_bs;
+      g.B = B.X[cur]; g.ldb = L.ld_m; g.b_bs = B.x_bs; g.b_kmajor = 0;
+      g.in_dtype = xdt;
+      g.D = B.X[1 - cur]; g.ldd = L.ld_m; g.d_bs = B.x_bs; g.d_dtype = xdt;
+      g.C = B.X[cur]; g.ldc = L.ld_m; g.c_bs = B.x_bs; g.c_dtype = xdt;
+      g.c_acc = coefB; g.c_in = a;
+      g.scale = B.inv; g.scale_pow = first ? 1 : 0;
+      if ((rc = gemm(c, g))) return rc;
+      cur = 1 - cur;
+    }
+    *out_x = cur;
+    return 0;
+  }
+
+  // ---------------------------------------------------------------- Gram forms
+  const bool stabilized = ns->mode == MUON_NS_GRAM_STABILIZED;
+  int x0 = 0;              // X buffer holding the matrix the Gram iteration applies to
+  bool x0_raw = true;      // still the unnormalised packed U (scale by inv on use)
+  void* R = B.S[0];
+  void* T = B.S[1];
+  void* Qbuf[3] = {B.S[2], B.S[3], B.S[4]};
+  int q_acc = -1;          // index into Qbuf, -1 = identity
+
+  auto gram_of_x = [&](bool raw) -> int {
+    GemmDesc g = desc(n, n, m, chunk);
+    g.A = B.X[x0]; g.lda = L.ld_m; g.a_bs = B.x_bs;
+    g.B = B.X[x0]; g.ldb = L.ld_m; g.b_bs = B.x_bs; g.b_kmajor = 1;
+    g.in_dtype = xdt;
+    g.D = R; g.ldd = L.ld_n; g.d_bs = B.s_bs; g.d_dtype = gdt;
+    g.scale = B.inv; g.scale_pow = raw ? 2 : 0;
+    g.symmetric = 1;
+    return gemm(c, g);
+  };
+  auto sq = [&](GemmDesc& g, const void* A, const void* Bop, int b_kmajor, void* D, int ddt) {
+    g = desc(n, n, n, chunk);
+    g.A = A; g.lda = L.ld_n; g.a_bs = B.s_bs;
+    g.B = Bop; g.ldb = L.ld_n; g.b_bs = B.s_bs; g.b_kmajor = b_kmajor;
+    g.in_dtype = gdt;
+    g.D = D; g.ldd = L.ld_n; g.d_bs = B.s_bs; g.d_dtype = ddt;
+  };
+  auto apply = [&](int x_out) -> int {  // X[x_out] = f Q_acc X0
+    GemmDesc g = desc(n, m, n, chunk);
+    g.A = Qbuf[q_acc]; g.lda = L.ld_n; g.a_bs = B.s_bs;
+    g.B = B.X[x0]; g.ldb = L.ld_m; g.b_bs = B.x_bs; g.b_kmajor = 0;
+    g.in_dtype = xdt;
+    g.D = B.X[x_out]; g.ldd = L.ld_m; g.d_bs = B.x_bs; g.d_dtype = xdt;
+    g.scale = B.inv; g.scale_pow = x0_raw ? 1 : 0;
+    return gemm(c, g);
+  };
+
+  if ((rc = gram_of_x(true))) return rc;
+  for (int k = 1; k <= K; ++k) {
+    const float a = ns->coeffs[3 * (k - 1)], bb = ns->coeffs[3 * (k - 1) + 1], cc = ns->coeffs[3 * (k - 1) + 2];
+    const bool last = k == K;
+    const bool restart = stabilized && k == ns->restart_after && !last;
+    const bool to_apply = last || restart;
+    // Q = a I + b R + c R R, into a slot that is not Q_acc
+    int qi = 0;
+    while (qi == q_acc) ++qi;
+    const int q_dt = (q_acc < 0 && to_apply) ? xdt : gdt;
+    GemmDesc g;
+    sq(g, R, R, 1, Qbuf[qi], q_dt);
+    g.C = R; g.ldc = L.ld_n; g.c_bs = B.s_bs; g.c_dtype = gdt;
+    g.c_acc = cc; g.c_in = bb; g.c_eye = a;
+    g.symmetric = 1;
+    if ((rc = gemm(c, g))) return rc;
+    if (q_acc < 0) {
+      q_acc = qi;
+    } else {
+      // Q_acc <- Q Q_acc
+      int ni = 0;
+      while (ni == q_acc || ni == qi) ++ni;
+      const int n_dt = to_apply ? xdt : gdt;
+      sq(g, Qbuf[qi], Qbuf[q_acc], 0, Qbuf[ni], n_dt);
+      if ((rc = gemm(c, g))) return rc;
+      q_acc = ni;
+    }
+    if (last) break;
+    if (restart) {
+      const int x_new = 1 - x0;
+      if ((rc = apply(x_new))) return rc;
+      x0 = x_new;
+      x0_raw = false;
+      if ((rc = gram_of_x(false))) return rc;
+      q_acc = -1;
+    } else {
+      // R <- Q R Q  as T = Q R, R = T Q
+      sq(g, Qbuf[qi], R, 0, T, gdt);
+      if ((rc = gemm(c, g))) return rc;
+      sq(g, T, Qbuf[qi], 0, R, gdt);
+      if ((rc = gemm(c, g))) return rc;
+    }
+  }
+  const int x_out = 1 - x0;
+  if ((rc = apply(x_out))) return rc;
+  *out_x = x_out;
+  return 0;
+}
+
+// ------------------------------------------------------------------ driver
+struct SrcView {      // what the pack / unpack kernels need for one caller group
+  int rows, cols;
+  int src_dtype, dst_dtype;
+  const void* const* src;
+  float* const* mom;
+  void* const* dst;
+};
+
+int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& views, const std::vector<long long>& first_index,
+                const muon_ns_params* ns, bool update, float mu, int nesterov, float lr, float wd, float scale_coef,
+                void* ws, size_t ws_bytes, int* status, cudaStream_t s) {
+  for (const Batch& bt : batches) {
+    const Layout L = make_layout(bt.n, bt.m, ns);
+    if (ws_bytes < chunk_bytes(L, 1)) return MUON_ERR_WORKSPACE;
+    const int chunk_cap = (int)std::min<size_t>((size_t)bt.total, (ws_bytes - L.fixed) / L.per_matrix);
+    // slots are assigned in segment order; walk them chunk by chunk
+    int seg_i = 0, seg_off = 0;
+    int done = 0;
+    while (done < bt.total) {
+      const int chunk = std::min(chunk_cap, bt.total - done);
+      const Bufs B = carve(L, chunk, ws);
+      if (cudaMemsetAsync(B.err, 0, sizeof(int), s) != cudaSuccess) return MUON_ERR_CUDA;
+      // pieces of segments covering slots [done, done + chunk)
+      struct Piece { int group, first, count, slot; };
+      std::vector<Piece> pieces;
+      {
+        int slot = 0, si = seg_i, so = seg_off;
+        while (slot < chunk) {
+          const Seg& sg = bt.segs[si];
+          int take = std::min(sg.count - so, chunk - slot);
+          int left = take, f = sg.first + so, sl = slot;
+          while (left > 0) {
+            const int t = std::min(left, SegmentPtrs::kMax);
+            pieces.push_back(Piece{sg.group, f, t, sl});
+            f += t; sl += t; left -= t;
+          }
+          slot += take;
+          so += take;
+          if (so == sg.count) { ++si; so = 0; }
+        }
+        seg_i = si;
+        seg_off = so;
+      }
+      const int xdt = ns->compute_dtype;
+      for (const Piece& pc : pieces) {
+        const SrcView& v = views[pc.group];
+        SegmentPtrs ptrs;
+        for (int i = 0; i < pc.count; ++i) {
+          ptrs.src[i] = v.src[pc.first + i];
+          ptrs.mom[i] = v.mom ? v.mom[pc.first + i] : nullptr;
+          ptrs.dst[i] = nullptr;
+        }
+        PackArgs a{};
+        a.rows = v.rows; a.cols = v.cols; a.count = pc.count;
+        a.src_dtype = v.src_dtype; a.x_dtype = xdt;
+        a.momentum_mode = update ? 1 : 0; a.mu = mu; a.nesterov = nesterov;
+        a.x = reinterpret_cast<char*>(B.X[0]) + (size_t)pc.slot * B.x_bs * L.x_es;
+        a.ld_x = L.ld_m; a.x_batch_stride = B.x_bs;
+        a.partials = B.partials + (size_t)pc.slot * L.tiles;
+        a.partial_stride = L.tiles;
+        launch_pack(a, ptrs, s);
+      }
+      launch_norm(B.partials, L.tiles, L.tiles, chunk, ns->eps, B.inv, s);
+      if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+      Ctx ctx{ns->compute_dtype, s, B.err};
+      int xi = 0;
+      if (run_chain(ctx, L, B, chunk, ns, &xi) != 0) return MUON_ERR_CUDA;
+      for (const Piece& pc : pieces) {
+        const SrcView& v = views[pc.group];
+        SegmentPtrs ptrs;
+        for (int i = 0; i < pc.count; ++i) {
+          ptrs.src[i] = nullptr;
+          ptrs.mom[i] = nullptr;
+          ptrs.dst[i] = v.dst[pc.first + i];
+        }
+        UnpackArgs u{};
+        u.rows = v.rows; u.cols = v.cols; u.count = pc.count;
+        u.dst_dtype = v.dst_dtype; u.x_dtype = xdt;
+        u.update_mode = update ? 1 : 0;
+        u.decay = 1.f - lr * wd;
+        u.step = lr * scale_coef * std::sqrt((float)std::max(v.rows, v.cols));
+        u.x = reinterpret_cast<const char*>(B.X[xi]) + (size_t)pc.slot * B.x_bs * L.x_es;
+        u.ld_x = L.ld_m; u.x_batch_stride = B.x_bs;
+        u.status = status ? status + first_index[pc.group] + pc.first : nullptr;
+        u.chunk_err = B.err;
+        launch_unpack(u, ptrs, s);
+      }
+      if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+      done += chunk;
+    }
+  }
+  return MUON_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int check_groups(const muon_group* groups, int n_groups, const muon_hparams* hp, long long* total) {
+  if (!groups || n_groups <= 0 || !hp) return MUON_ERR_INVALID;
+  if (!ns_params_ok(&hp->ns)) return MUON_ERR_INVALID;
+  if (!std::isfinite(hp->lr) || !std::isfinite(hp->momentum) || !std::isfinite(hp->weight_decay) ||
+      !std::isfinite(hp->scale_coef))
+    return MUON_ERR_INVALID;
+  long long t = 0;
+  for (int g = 0; g < n_groups; ++g) {
+    const muon_group& G = groups[g];
+    if (G.rows <= 0 || G.cols <= 0 || G.count < 0) return MUON_ERR_INVALID;
+    if ((long long)G.rows * G.cols > (1LL << 34)) return MUON_ERR_INVALID;
+    if (!dtype_ok(G.w_dtype) || !dtype_ok(G.g_dtype)) return MUON_ERR_UNSUPPORTED;
+    if (G.count > 0 && (!G.W || !G.G || !G.M)) return MUON_ERR_INVALID;
+    for (int i = 0; i < G.count; ++i) {
+      if (!G.W[i] || !G.G[i] || !G.M[i]) return MUON_ERR_INVALID;
+      if (!aligned16(G.W[i]) || !aligned16(G.G[i]) || !aligned16(G.M[i])) return MUON_ERR_INVALID;
+    }
+    t += G.count;
+  }
+  *total = t;
+  return MUON_OK;
+}
+
+size_t ws_for(const std::vector<Batch>& batches, const muon_ns_params* ns, bool full) {
+  size_t best = 0;
+  for (const Batch& b : batches) {
+    const Layout L = make_layout(b.n, b.m, ns);
+    best = std::max(best, chunk_bytes(L, full ? b.total : 1));
+  }
+  return best;
+}
+
+double flops_of(int rows, int cols, const muon_ns_params* ns) {
+  const double n = std::min(rows, cols), m = std::max(rows, cols);
+  const double sq = 2.0 * m * n * n, cube = 2.0 * n * n * n;
+  const int K = ns->iters;
+  if (ns->mode == MUON_NS_STANDARD) {
+    double per = sq + sq;  // X X^T and B X
+    double total = 0;
+    for (int k = 0; k < K; ++k) total += per + (ns->coeffs[3 * k + 2] != 0.f ? cube : 0.0);
+    return total;
+  }
+  // Gram forms: R0, per iteration R^2 (+ Q Q_acc unless Q_acc = I), R update
+  // (2 products) or the restart pair, final apply
+  double total = sq;
+  bool fresh = true;
+  for (int k = 1; k <= K; ++k) {
+    total += cube;
+    if (!fresh) total += cube;
+    fresh = false;
+    if (k == K) break;
+    if (ns->mode == MUON_NS_GRAM_STABILIZED && k == ns->restart_after) {
+      total += 2 * sq;
+      fresh = true;
+    } else {
+      total += 2 * cube;
+    }
+  }
+  return total + sq;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t muon_workspace_size(const muon_group* groups, int n_groups, const muon_hparams* hp) {
+  long long total = 0;
+  if (check_groups(groups, n_groups, hp, &total) != MUON_OK) return 0;
+  return ws_for(plan_groups(groups, n_groups), &hp->ns, true);
+}
+
+size_t muon_workspace_min(const muon_group* groups, int n_groups, const muon_hparams* hp) {
+  long long total = 0;
+  if (check_groups(groups, n_groups, hp, &total) != MUON_OK) return 0;
+  return ws_for(plan_groups(groups, n_groups), &hp->ns, false);
+}
+
+int muon_step(const muon_group* groups, int n_groups, const muon_hparams* hp, void* ws, size_t ws_bytes,
+              int* status_per_matrix, void* stream) {
+  long long total = 0;
+  int rc = check_groups(groups, n_groups, hp, &total);
+  if (rc != MUON_OK) return rc;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return MUON_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<Batch> batches = plan_groups(groups, n_groups);
+  if (ws_bytes < ws_for(batches, &hp->ns, false)) return MUON_ERR_WORKSPACE;
+  std::vector<SrcView> views(n_groups);
+  std::vector<long long> first(n_groups);
+  long long acc = 0;
+  for (int g = 0; g < n_groups; ++g) {
+    views[g] = SrcView{groups[g].rows, groups[g].cols, groups[g].g_dtype, groups[g].w_dtype,
+                       groups[g].G, groups[g].M, groups[g].W};
+    first[g] = acc;
+    acc += groups[g].count;
+  }
+  if (status_per_matrix && total > 0 && cudaMemsetAsync(status_per_matrix, 0, (size_t)total * sizeof(int), s) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  return run_batches(batches, views, first, &hp->ns, true, hp->momentum, hp->nesterov, hp->lr, hp->weight_decay,
+                     hp->scale_coef, ws, ws_bytes, status_per_matrix, s);
+}
+
+size_t muon_ns_workspace_size(int count, int rows, int cols, const muon_ns_params* ns) {
+  if (count <= 0 || rows <= 0 || cols <= 0 || !ns_params_ok(ns)) return 0;
+  const Layout L = make_layout(std::min(rows, cols), std::max(rows, cols), ns);
+  return chunk_bytes(L, count);
+}
+
+int muon_ns_batched(void* const* X, int count, int rows, int cols, int dtype, const muon_ns_params* ns, void* ws,
+                    size_t ws_bytes, int* status_per_matrix, void* stream) {
+  if (!X || count < 0 || rows <= 0 || cols <= 0 || !ns_params_ok(ns)) return MUON_ERR_INVALID;
+  if ((long long)rows * cols > (1LL << 34)) return MUON_ERR_INVALID;
+  if (!dtype_ok(dtype)) return MUON_ERR_UNSUPPORTED;
+  if (count == 0) return MUON_OK;
+  for (int i = 0; i < count; ++i)
+    if (!X[i] || !aligned16(X[i])) return MUON_ERR_INVALID;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1))) return MUON_ERR_INVALID;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Batch b{std::min(rows, cols), std::max(rows, cols), {Seg{0, 0, count}}, count};
+  std::vector<Batch> batches{b};
+  if (ws_bytes < ws_for(batches, ns, false)) return MUON_ERR_WORKSPACE;
+  std::vector<SrcView> views{SrcView{rows, cols, dtype, dtype, const_cast<const void* const*>(X), nullptr, X}};
+  std::vector<long long> first{0};
+  if (status_per_matrix && cudaMemsetAsync(status_per_matrix, 0, (size_t)count * sizeof(int), s) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  return run_batches(batches, views, first, ns, false, 0.f, 0, 0.f, 0.f, 0.f, ws, ws_bytes, status_per_matrix, s);
+}
+
+double muon_ns_flops(int rows, int cols, const muon_ns_params* ns) {
+  if (rows <= 0 || cols <= 0 || !ns_params_ok(ns)) return 0.0;
+  return flops_of(rows, cols, ns);
+}
+
+const char* muon_status_string(int code) {
+  switch (code) {
+    case MUON_OK: return "ok";
+    case MUON_ERR_INVALID: return "invalid argument (null or misaligned pointer, bad shape, count or parameter)";
+    case MUON_ERR_UNSUPPORTED: return "unsupported dtype";
+    case MUON_ERR_WORKSPACE: return "workspace too small";
+    case MUON_ERR_CUDA: return "CUDA launch or tensor-map encode failed";
+    case MUON_STATUS_NONFINITE: return "non-finite values in the orthogonalised matrix";
+    case MUON_STATUS_TIMEOUT: return "a device-side wait timed out; the matrix was not finished";
+    case MUON_STATUS_NONFINITE | MUON_STATUS_TIMEOUT: return "non-finite values and a device-side wait timeout";
+    default: return "unknown code";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,560 @@
+// Tensor-core product for the Newton-Schulz chain on sm_100a (tcgen05 + TMEM + TMA).
+//
+// Every product of the iteration ("Gram Newton-Schulz" write-up: X X^T, A^2,
+// B X; and the Gram form's R^2, Q Q_acc, Q R Q, Q_acc X_0) is one launch of
+// this kernel over a batch of same-shape matrices:
+//
+//   D[b] = f_b * (c_acc * A[b] op(B[b]) + c_in * C[b]) + c_eye * I
+//
+// with f_b = scale[b]^p carrying the Frobenius normalisation into the first
+// products (so the packed X_0 never has to be rescaled in memory), C the
+// polynomial's linear term (b A, b R) or the a X term, and c_eye the a I of
+// Q = a I + b R + c R^2.  Symmetric results (X X^T, A A, R R) are computed on
+// the upper-triangle 128 x 128 blocks only and mirrored on store.
+//
+// Structure (one CTA per SM, persistent over the batch's tiles):
+//   warp 0        TMA producer: 128x64 A tile + 256x64 B tile per stage,
+//                 128-byte swizzle, STAGES-deep ring of shared-memory slots
+//   warp 1        TMEM allocator + single-thread tcgen05.mma issuer
+//                 (M=128, N=256, K=16 per instruction, fp32 accumulate)
+//   warps 2..5    epilogue: tcgen05.ld of the accumulator (one TMEM lane =
+//                 one output row per thread), polynomial epilogue, stores
+//   TMEM holds two 128x256 fp32 accumulators so the epilogue of tile i
+//   overlaps the main loop of tile i+1.
+// Every mbarrier wait is bounded (global-timer deadline plus a CTA-wide abort
+// flag); on expiry the CTA drains its in-flight copies and MMAs, frees TMEM,
+// raises the timeout bit in the caller's error word and returns.
+#include <cuda.h>
+#include <stdio.h>
+#include <stdlib.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace muon {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;                   // 64 x 2 B = one 128-byte swizzle row
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int B_BYTES = BN * BK * 2;     // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr int TMEM_COLS = 2 * BN;        // two fp32 accumulators
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int GROUP_M = 8;               // tile raster grouping for L2 reuse
+
+struct Params {
+  int M, N, K, batch;
+  int tiles_m, tiles_n, tiles_per_batch, total_tiles;
+  int symmetric;
+  void* D; int ldd; long long d_bs; int d_dtype;
+  const void* C; int ldc; long long c_bs; int c_dtype;
+  float c_acc, c_in, c_eye;
+  const float* scale; int scale_pow;
+  int* err;
+  long long timeout_ns;
+};
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the deadline passed or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if ((long long)(global_timer() - t0) > timeout_ns) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor for kind::f16: fp32 D, A/B of one 16-bit type,
+// A K-major, B K-major or MN-major, M = 128, N = 256.
+__host__ __device__ constexpr uint32_t make_idesc(int in_fmt /*0 f16, 1 bf16*/, int b_mn) {
+  return (1u << 4) | ((uint32_t)in_fmt << 7) | ((uint32_t)in_fmt << 10) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ tile order
+struct Tile { int b, tm, tn; };
+
+__device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
+  Tile r;
+  r.b = t / p.tiles_per_batch;
+  int q = t - r.b * p.tiles_per_batch;
+  if (p.symmetric) {
+    // upper-triangle tiles in 128-block units: row tm keeps tn >= tm / 2
+    int tm = 0;
+    for (; tm < p.tiles_m; ++tm) {
+      const int cnt = p.tiles_n - tm / 2;
+      if (q < cnt) break;
+      q -= cnt;
+    }
+    r.tm = tm;
+    r.tn = tm / 2 + q;
+  } else {
+    const int per_group = GROUP_M * p.tiles_n;
+    const int g = q / per_group;
+    const int first = g * GROUP_M;
+    const int gsz = min(p.tiles_m - first, GROUP_M);
+    const int w = q - g * per_group;
+    r.tm = first + w % gsz;
+    r.tn = w / gsz;
+  }
+  return r;
+}
+
+// ------------------------------------------------------------------ epilogue
+__device__ __forceinline__ void store_row32(void* D, int dt, long long off, const float* v) {
+  uint4 q[4];
+  if (dt == kBF16) {
+    __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) e[i] = __float2bfloat16_rn(v[i]);
+    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(D) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = q[i];
+  } else {
+    __half* e = reinterpret_cast<__half*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) e[i] = __float2half_rn(v[i]);
+    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(D) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = q[i];
+  }
+}
+
+__device__ __forceinline__ void load_row32(const void* C, int dt, long long off, float* v) {
+  uint4 q[4];
+  const uint4* s = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(C) + off * 2);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q[i] = s[i];
+  if (dt == kBF16) {
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(e[i]);
+  } else {
+    const __half* e = reinterpret_cast<const __half*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __half2float(e[i]);
+  }
+}
+
+__device__ __forceinline__ void epilogue_chunk(const Params& p, const Tile& t, int row_in_tile, int chunk,
+                                               const uint32_t (&acc)[32], float f) {
+  const int gi = t.tm * BM + row_in_tile;
+  const int gj0 = t.tn * BN + chunk * 32;
+  bool mirror = false;
+  if (p.symmetric) {
+    const int bj = t.tn * 2 + (chunk >> 2);  // 128-column block of this chunk
+    if (bj < t.tm) return;                   // lower block: its mirror is stored elsewhere
+    mirror = bj > t.tm;
+  }
+  if (gi >= p.M || gj0 >= p.N) return;
+  const bool full = (gj0 + 32 <= p.N);
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = p.c_acc * __uint_as_float(acc[j]);
+  if (p.C != nullptr) {
+    const char* cb = reinterpret_cast<const char*>(p.C) + (long long)t.b * p.c_bs * 2;
+    const long long off = (long long)gi * p.ldc + gj0;
+    if (full) {
+      float c[32];
+      load_row32(cb, p.c_dtype, off, c);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += p.c_in * c[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (gj0 + j < p.N) v[j] += p.c_in * load_any(cb, off + j, p.c_dtype);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    v[j] *= f;
+    if (gj0 + j == gi) v[j] += p.c_eye;
+  }
+
+  char* db = reinterpret_cast<char*>(p.D) + (long long)t.b * p.d_bs * 2;
+  {
+    const long long off = (long long)gi * p.ldd + gj0;
+    if (full) {
+      store_row32(db, p.d_dtype, off, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (gj0 + j < p.N) store_any(db, off + j, p.d_dtype, v[j]);
+    }
+  }
+  if (mirror) {
+    // D[gj][gi]: for each j the warp's 32 rows form 32 consecutive columns.
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (gj0 + j < p.N) store_any(db, (long long)(gj0 + j) * p.ldd + gi, p.d_dtype, v[j]);
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <bool B_MN, int IN_FMT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+            const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full_bar = bars;                    // [STAGES]
+  uint64_t* empty_bar = bars + STAGES;          // [STAGES]
+  uint64_t* tfull_bar = bars + 2 * STAGES;      // [2]
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2; // [2]
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;  // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull_bar[a]), 1);
+      mbar_init(smem_u32(&tempty_bar[a]), 128);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) issued[s] = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile(p, t);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&full_bar[stage]);
+          mbar_expect_tx(fb, STAGE_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+          tma_load_3d(sa, &tmap_a, fb, kb * BK, tl.tm * BM, tl.b);
+          if (B_MN) {
+#pragma unroll
+            for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * (BK * 128), &tmap_b, fb, tl.tn * BN + q * 64, kb * BK, tl.b);
+          } else {
+            tma_load_3d(sb, &tmap_b, fb, kb * BK, tl.tn * BN, tl.b);
+          }
+          issued[stage]++;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // drain: every stage's most recent load must land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued[s]) {
+            volatile int never = 0;
+            mbar_wait(smem_u32(&full_bar[s]), (issued[s] - 1) & 1u, &never, p.timeout_ns);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc(IN_FMT, B_MN ? 1 : 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.total_tiles && ok; t += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(smem_u32(&tempty_bar[acc]), aph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            const uint64_t ad = smem_desc(sa + k * (UMMA_K * 2), 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc(sb + k * (UMMA_K * 128), BK * 128, 1024)
+                                     : smem_desc(sb + k * (UMMA_K * 2), 16, 1024);
+            tc_mma(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          tc_commit(smem_u32(&empty_bar[stage]));  // slot free once these MMAs retire
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&tfull_bar[acc]));      // accumulator ready for the epilogue
+      }
+      // all issued MMAs retire before TMEM is released
+      tc_commit(smem_u32(drain_bar));
+      volatile int never = 0;
+      mbar_wait(smem_u32(drain_bar), 0, &never, p.timeout_ns);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
+      const Tile tl = decode_tile(p, t);
+      const int acc = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(smem_u32(&tfull_bar[acc]), aph, abort_flag, p.timeout_ns);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const float f = matrix_scale(p.scale, p.scale_pow, tl.b);
+      const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + (uint32_t)(c * 32), r);
+        if (c == BN / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(smem_u32(&tempty_bar[acc]));
+        }
+        epilogue_chunk(p, tl, row_in_tile, c, r, f);
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+  if (threadIdx.x == 0 && *abort_flag && p.err != nullptr) atomicOr(p.err, kStatusTimeout);
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D tiled map over a batch of row-major matrices: dims (inner, outer, batch).
+static bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer,
+                       long long batch, long long ld_elems, long long bs_elems, int box_inner, int box_outer) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  const CUtensorMapDataType dt = dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)batch};
+  cuuint64_t strides[2] = {(cuuint64_t)ld_elems * 2, (cuuint64_t)(bs_elems > 0 ? bs_elems : ld_elems * outer) * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool B_MN, int IN_FMT>
+static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<B_MN, IN_FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return (int)e;
+    attr_done = true;
+  }
+  const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
+  gemm_kernel<B_MN, IN_FMT><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace tc
+
+int gemm_tc(const GemmDesc& g, cudaStream_t s) {
+  using namespace tc;
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return 0;
+  if (g.in_dtype != kBF16 && g.in_dtype != kFP16) return (int)cudaErrorInvalidValue;
+  if (g.d_dtype == kFP32 || (g.C && g.c_dtype == kFP32)) return (int)cudaErrorInvalidValue;
+  if (g.symmetric && g.M != g.N) return (int)cudaErrorInvalidValue;
+  Params p{};
+  p.M = g.M; p.N = g.N; p.K = g.K; p.batch = g.batch;
+  p.tiles_m = (g.M + BM - 1) / BM;
+  p.tiles_n = (g.N + BN - 1) / BN;
+  if (g.symmetric) {
+    int cnt = 0;
+    for (int tm = 0; tm < p.tiles_m; ++tm) cnt += p.tiles_n - tm / 2;
+    p.tiles_per_batch = cnt;
+  } else {
+    p.tiles_per_batch = p.tiles_m * p.tiles_n;
+  }
+  long long total = (long long)p.tiles_per_batch * g.batch;
+  if (total > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
+  p.total_tiles = (int)total;
+  p.symmetric = g.symmetric;
+  p.D = g.D; p.ldd = g.ldd; p.d_bs = g.d_bs; p.d_dtype = g.d_dtype;
+  p.C = g.C; p.ldc = g.ldc; p.c_bs = g.c_bs; p.c_dtype = g.c_dtype;
+  p.c_acc = g.c_acc; p.c_in = g.c_in; p.c_eye = g.c_eye;
+  p.scale = g.scale; p.scale_pow = g.scale_pow;
+  p.err = g.err;
+  p.timeout_ns = wait_timeout_ns();
+
+  CUtensorMap ma, mb;
+  if (!encode_map(&ma, g.in_dtype, g.A, g.K, g.M, g.batch, g.lda, g.a_bs, BK, BM)) return (int)cudaErrorInvalidValue;
+  const bool bmn = !g.b_kmajor;
+  if (bmn) {
+    if (!encode_map(&mb, g.in_dtype, g.B, g.N, g.K, g.batch, g.ldb, g.b_bs, 64, BK)) return (int)cudaErrorInvalidValue;
+  } else {
+    if (!encode_map(&mb, g.in_dtype, g.B, g.K, g.N, g.batch, g.ldb, g.b_bs, BK, BN)) return (int)cudaErrorInvalidValue;
+  }
+  const int fmt = g.in_dtype == kBF16 ? 1 : 0;
+  if (bmn) return fmt ? launch<true, 1>(ma, mb, p, s) : launch<true, 0>(ma, mb, p, s);
+  return fmt ? launch<false, 1>(ma, mb, p, s) : launch<false, 0>(ma, mb, p, s);
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+long long wait_timeout_ns() {
+  static long long ns = -1;
+  if (ns < 0) {
+    const char* e = getenv("MUON_WAIT_TIMEOUT_MS");
+    long long ms = e ? atoll(e) : 4000;
+    if (ms <= 0) ms = 4000;
+    ns = ms * 1000000LL;
+  }
+  return ns;
+}
+
+}  // namespace muon

@@ -1,0 +1,87 @@
+// Internal launchers shared between the translation units of libmuon.
+// Nothing here is part of the C ABI (see include/muon.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace muon {
+
+// ---------------------------------------------------------------- elementwise
+// One "segment" = `count` matrices of one storage shape rows x cols that land
+// in consecutive slots [slot0, slot0 + count) of an oriented n x m workspace
+// batch (n = min, m = max; a tall matrix is transposed on the way in and out).
+struct SegmentPtrs {
+  static constexpr int kMax = 256;  // matrices per launch (kernel-parameter space)
+  const void* src[kMax];  // G (momentum mode) or X (copy mode)
+  float* mom[kMax];       // M (momentum mode only)
+  void* dst[kMax];        // W (update mode) or X (copy mode)
+};
+
+struct PackArgs {
+  int rows, cols, count;
+  int src_dtype;        // G or X storage dtype
+  int x_dtype;          // workspace dtype (bf16/fp16 tensor path, fp32 SIMT path)
+  int momentum_mode;    // 1: M <- mu M + (1-mu) G, U = nesterov ? lerp : M;  0: U = src
+  float mu;
+  int nesterov;
+  void* x;              // workspace X batch, slot0 already applied
+  int ld_x;             // leading dimension of X (>= m)
+  long long x_batch_stride;
+  float* partials;      // [count][tiles] sums of squares, slot0 applied
+  int partial_stride;   // partial entries per matrix
+};
+int pack_tiles(int rows, int cols);
+void launch_pack(const PackArgs& a, const SegmentPtrs& p, cudaStream_t s);
+
+// inv[b] = 1 / (sqrt(sum partials[b][:]) + eps), deterministic order.
+void launch_norm(const float* partials, int partial_stride, int n_partials, int count,
+                 float eps, float* inv, cudaStream_t s);
+
+struct UnpackArgs {
+  int rows, cols, count;
+  int dst_dtype;        // W or X storage dtype
+  int x_dtype;
+  int update_mode;      // 1: W <- decay W - step O;  0: X <- O
+  float decay, step;    // decay = 1 - lr wd, step = lr * scale_coef * sqrt(max(r,c))
+  const void* x;        // oriented result batch, slot0 applied
+  int ld_x;
+  long long x_batch_stride;
+  int* status;          // per-matrix status words for these matrices (may be null)
+  const int* chunk_err; // device word with errors raised by the chunk's GEMMs (may be null)
+};
+void launch_unpack(const UnpackArgs& a, const SegmentPtrs& p, cudaStream_t s);
+
+// Fill n x n identity-free helpers
+void launch_convert(const void* src, int src_dtype, void* dst, int dst_dtype, long long n,
+                    cudaStream_t s);
+
+// ---------------------------------------------------------------- products
+// D[b] = epilogue(A[b] * op(B[b])) for b < batch, all row-major.
+//   A is M x K (K contiguous).  op(B) is K x N given either as rows of
+//   length K (b_kmajor = 1: B stored N x K, i.e. D = A B^T) or as rows of
+//   length N (b_kmajor = 0: B stored K x N, D = A B).
+//   epilogue: out = f*(c_acc*acc + c_in*Cin) + (row == col ? c_eye : 0),
+//   f = scale[b]^scale_pow.  symmetric = 1 asks for the upper-triangle tiles
+//   only (M == N, result known symmetric), mirrored on store.
+struct GemmDesc {
+  int M, N, K, batch;
+  const void* A; int lda; long long a_bs;
+  const void* B; int ldb; long long b_bs; int b_kmajor;
+  int in_dtype;           // operand dtype (A and B share it)
+  void* D; int ldd; long long d_bs; int d_dtype;
+  const void* C; int ldc; long long c_bs; int c_dtype;  // optional Cin
+  float c_acc, c_in, c_eye;
+  const float* scale; int scale_pow;
+  int symmetric;
+  int* err;               // device word: timeout bits land here (may be null)
+};
+// Tensor-core (tcgen05) path: bf16/fp16 operands.  Returns 0 or a CUDA error.
+int gemm_tc(const GemmDesc& g, cudaStream_t s);
+// SIMT path (any dtype, fp32 math): used for fp32 compute.
+int gemm_simt(const GemmDesc& g, cudaStream_t s);
+
+int num_sms();
+long long wait_timeout_ns();
+
+}  // namespace muon
