@@ -1,0 +1,392 @@
+#!/usr/bin/env python
+"""Benchmark: one Muon optimizer step (momentum, Nesterov, Frobenius
+normalisation, five quintic Newton-Schulz iterations, update scaling and
+decoupled weight decay) over the Kimi-K2-shaped parameter set on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload kimi-k2|dense|moe|single] [--mode standard|gram|gram_stabilized]
+
+A step is one muon_step call over all matrices of the workload (inputs resident
+in HBM).  The metric is effective TFLOP/s: the iteration's algorithmic FLOPs
+(every product 2 * rows * cols * inner, 4 m n^2 + 2 n^3 per standard
+iteration, as the Gram Newton-Schulz write-up counts them) divided by the
+device time of the step; ms per step is reported beside it.  Multi-GPU runs
+(torchrun, one process per GPU) give every rank its own full parameter set
+(weak scaling, no collective on the data path); the step time is the max over
+ranks.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload (one expert matrix per step) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "NS-orthogonalization ms/optimizer-step & effective TFLOP/s (% of bf16 peak)"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["kimi-k2", "kimi-k2-experts16", "dense", "moe", "single"], default="kimi-k2",
+                   help="kimi-k2-experts16: 16 expert matrices of the K2 set (small case for profiling)")
+    p.add_argument("--mode", choices=["standard", "gram", "gram_stabilized"], default="standard")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-compare", action="store_true", help="skip the stabilised-Gram comparison run")
+    p.add_argument("--workspace-gb", type=float, default=24.0, help="workspace cap (chunks the step beyond it)")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def build_workload(name, device):
+    import synth
+    if name == "kimi-k2":
+        w = synth.kimi_k2(device=device)
+    elif name == "kimi-k2-experts16":
+        w = synth.kimi_k2(device=device, counts=[16, 0, 0, 0])
+    elif name == "dense":
+        w = synth.dense_projection(device=device)
+    elif name == "moe":
+        w = synth.moe_layer(device=device)
+    else:
+        w = synth.single_fp32(device=device)
+    params, grads, moms = [], [], []
+    for g in w.groups:
+        params += g.W
+        grads += g.G
+        moms += g.M
+    return w, params, grads, moms
+
+
+def workload_config(w, params, mode, steps_note):
+    shapes = {}
+    for p in params:
+        k = "x".join(map(str, p.shape))
+        shapes[k] = shapes.get(k, 0) + 1
+    return {"workload": w.name, "matrices": len(params), "shapes": shapes, "mode": mode,
+            "ns_iters": 5, "coeffs": [3.4445, -4.7750, 2.0315], "momentum": 0.95, "nesterov": True, "lr": 0.02,
+            "weight_decay": 0.1, "scale_coef": 0.2, "l2": steps_note, "parallelism": "replicas (weak)"}
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling during the timed region."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.uuid = None
+        try:
+            u = str(torch.cuda.get_device_properties(device).uuid)
+            self.uuid = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            pass
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        rows = []
+        for line in open(self.file.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            if self.uuid and parts[0] != self.uuid:
+                continue
+            rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+        sm = [num(r[1]) for r in rows]
+        mx = max(num(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(num(r[3]) for r in rows)}
+
+
+def roofline_from_profile(prof, peaks, peak_kind):
+    gemm = [r for r in prof if r["kernel"].startswith("gemm_kernel")]
+    if not gemm:
+        return None
+    fl = sum(r["flops"] for r in gemm)
+    ms = sum(r["ms"] for r in gemm)
+    n = sum(r["launches"] for r in gemm)
+    achieved = fl / (ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
+    return {"bound": "tensor", "kernel": "gemm_kernel (tcgen05, all launches of the step)",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
+            "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
+            "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n, "traffic": None}
+
+
+def cpu_baseline_sample(w, hp, budget_s=20.0):
+    """Time the fp64 oracle on whole expert matrices until ~budget_s of CPU work."""
+    import numpy as np
+    import oracle
+    from threadpoolctl import threadpool_info
+    g = w.groups[0]
+    done_flops = 0.0
+    t0 = time.perf_counter()
+    n = 0
+    while n < len(g.W):
+        W = g.W[n].double().cpu().numpy()
+        G = g.G[n].double().cpu().numpy()
+        M = g.M[n].double().cpu().numpy()
+        ts = time.perf_counter()
+        oracle.muon_step(W, G, M, lr=hp["lr"], momentum=hp["momentum"], nesterov=hp["nesterov"],
+                         weight_decay=hp["weight_decay"], scale_coef=hp["scale_coef"], eps=hp["eps"],
+                         coeffs=hp["coeffs"], mode=hp["mode"], restart_after=hp["restart_after"])
+        done_flops += oracle.flops(g.rows, g.cols, len(hp["coeffs"]), hp["mode"], hp["restart_after"])
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+        del W, G, M, ts
+    el = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": done_flops / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {len(g.W)} matrices of shape {g.rows}x{g.cols}, full Muon step in fp64 "
+                      f"({done_flops / 1e12:.2f} TFLOP in {el:.1f} s)"}
+
+
+def run_reference(args):
+    """--impl reference: the fp64 oracle on the host cores, one matrix per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    from threadpoolctl import threadpool_info
+    w = synth.kimi_k2(device="cpu", counts=[1, 0, 0, 0]) if args.workload == "kimi-k2" else build_workload(args.workload, "cpu")[0]
+    hp = dict(w.hp, mode=args.mode)
+    g = w.groups[0]
+    W = g.W[0].double().numpy(); G = g.G[0].double().numpy(); M = g.M[0].double().numpy()
+    def one():
+        oracle.muon_step(W, G, M, lr=hp["lr"], momentum=hp["momentum"], nesterov=hp["nesterov"],
+                         weight_decay=hp["weight_decay"], scale_coef=hp["scale_coef"], eps=hp["eps"],
+                         coeffs=hp["coeffs"], mode=hp["mode"], restart_after=hp["restart_after"])
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    el = (time.perf_counter() - t0) / max(args.steps, 1)
+    fl = oracle.flops(g.rows, g.cols, len(hp["coeffs"]), hp["mode"], hp["restart_after"])
+    value = fl / el / 1e12
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    sample = f"one {g.rows}x{g.cols} matrix per step (of the {w.name} set), full Muon step in fp64"
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "mode": hp["mode"], "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    import newton_schulz_matrix_b200 as nsm
+    peaks, peak_kind = load_peaks()
+    w, params, grads, moms = build_workload(args.workload, device)
+    hp = dict(w.hp, mode=args.mode)
+    compute = hp.get("compute_dtype", "bf16")
+    ws_cap = int(args.workspace_gb * (1 << 30))
+    step = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, lr=hp["lr"], momentum=hp["momentum"],
+                        nesterov=hp["nesterov"], weight_decay=hp["weight_decay"], scale_coef=hp["scale_coef"],
+                        eps=hp["eps"], coeffs=hp["coeffs"], mode=hp["mode"], restart_after=hp["restart_after"],
+                        compute_dtype=compute)
+    flops_step = sum(nsm.muon_ns_flops(p.shape[0], p.shape[1], coeffs=hp["coeffs"], mode=hp["mode"],
+                                       restart_after=hp["restart_after"]) for p in params)
+    resident = sum(t.numel() * t.element_size() for t in params + grads + moms)
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(device)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(device)
+    nsm.muon_profile_begin()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    prof = nsm.muon_profile_end()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if dist is not None:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    status = step.status.cpu()
+    value = world * flops_step / (ms / 1e3) / 1e12
+    launches_timed = sum(r["launches"] for r in prof)
+
+    # stabilised Gram comparison on the same matrices (context for the Gram-vs-standard claim)
+    compare = None
+    if not args.no_compare and args.mode == "standard" and compute != "fp32":
+        del step
+        torch.cuda.empty_cache()
+        st2 = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, lr=hp["lr"], momentum=hp["momentum"],
+                           nesterov=hp["nesterov"], weight_decay=hp["weight_decay"], scale_coef=hp["scale_coef"],
+                           eps=hp["eps"], coeffs=hp["coeffs"], mode="gram_stabilized", restart_after=2)
+        st2()
+        torch.cuda.synchronize(device)
+        barrier()
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nrep = max(2, args.steps // 2)
+        c0.record(stream)
+        for _ in range(nrep):
+            st2()
+        c1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        gms = c0.elapsed_time(c1) / nrep
+        if dist is not None:
+            t = torch.tensor([gms], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            gms = float(t.item())
+        compare = {"gram_stabilized_ms_per_step": round(gms, 3), "standard_ms_per_step": round(ms, 3),
+                   "speedup_vs_standard": round(ms / gms, 3)}
+        step = st2
+
+    # end to end through the public API: gradients H2D from pinned host memory,
+    # the step, updated weights D2H to pinned host memory, every step
+    e2e = None
+    if not args.no_e2e:
+        hG = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
+        hW = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
+        for h, g in zip(hG, grads):
+            h.copy_(g)
+        e2e_step = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, lr=hp["lr"], momentum=hp["momentum"],
+                                nesterov=hp["nesterov"], weight_decay=hp["weight_decay"], scale_coef=hp["scale_coef"],
+                                eps=hp["eps"], coeffs=hp["coeffs"], mode=hp["mode"],
+                                restart_after=hp["restart_after"], compute_dtype=compute)
+        del step
+        torch.cuda.synchronize(device)
+        barrier()
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(args.e2e_steps):
+            for d, h in zip(grads, hG):
+                d.copy_(h, non_blocking=True)
+            e2e_step()
+            for h, d in zip(hW, params):
+                h.copy_(d, non_blocking=True)
+        x1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        ems = x0.elapsed_time(x1) / args.e2e_steps
+        if dist is not None:
+            t = torch.tensor([ems], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * flops_step / (ems / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": round(ems, 3),
+               "h2d_bytes_per_step": sum(g.numel() * g.element_size() for g in grads),
+               "d2h_bytes_per_step": sum(p.numel() * p.element_size() for p in params)}
+        del hG, hW
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(w, hp)
+
+    if rank == 0:
+        roof = roofline_from_profile(prof, peaks, peak_kind)
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if compute != "fp32" else "f32",
+            "data": "synthetic (seeded recipes of the workload; no datasets)",
+            "config": workload_config(w, params, hp["mode"], f"inputs larger than L2 ({resident / 2**30:.1f} GiB resident)"),
+            "pct_of_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
+            "peaks": {"bf16_tflops": peaks["bf16_tflops"], "bf16_tflops_sustained": peaks.get("bf16_tflops_sustained"),
+                      "source": peak_kind},
+            "flops_per_step": flops_step,
+            "clocks": clk, "e2e": e2e, "gpu_launches": launches_timed, "roofline": roof, "cpu_baseline": cpu,
+            "kernels": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()} for r in prof],
+            "status_nonzero": int((status != 0).sum()),
+        }
+        if compare:
+            line["compare"] = compare
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

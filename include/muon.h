@@ -74,10 +74,12 @@ enum {
  *                  matrix is rebuilt (1 <= restart_after < iters; 2 in [GramNS])
  *   eps            X0 = U / (||U||_F + eps)  [Moonlight, NS section; listing eps]
  *   compute_dtype  MUON_BF16 or MUON_FP16: tcgen05 tensor cores, fp32
- *                  accumulate, 16-bit storage between products;
- *                  MUON_FP32: CUDA-core FFMA products in fp32 throughout
- *   gram_dtype     Gram modes: storage of R, Q, Q_acc (MUON_FP16 or MUON_BF16;
- *                  ignored for FP32 compute and STANDARD) */
+ *                  accumulate, 16-bit storage of X, A, B between the products
+ *                  of the standard form; MUON_FP32: CUDA-core FFMA products in
+ *                  fp32 throughout (any mode)
+ *   gram_dtype     Gram modes on tensor cores: the 16-bit type of every matrix
+ *                  the Gram chain stores (R, Q, Q_acc, X0 and the restart X),
+ *                  MUON_FP16 (the stabilised variant's float16) or MUON_BF16 */
 typedef struct {
   int iters;
   const float* coeffs;
@@ -142,6 +144,25 @@ MUON_API int muon_ns_batched(void* const* X, int count, int rows, int cols, int 
 /* Algorithmic FLOPs of one orthogonalisation of a rows x cols matrix, every
  * product counted as 2 * rows * cols * inner [GramNS cost list]. */
 MUON_API double muon_ns_flops(int rows, int cols, const muon_ns_params* ns);
+
+/* Opt-in launch profiler (tracing aid).  Between muon_profile_begin() and
+ * muon_profile_end(), every kernel the library launches is bracketed by a pair
+ * of CUDA events recorded on the launch stream; this is the only state the
+ * library keeps between calls, and only while profiling is on.
+ * muon_profile_end synchronises on those events and fills up to max_entries
+ * rows, one per kernel kind that ran: its name, launch count, summed device
+ * time, and the algorithmic FLOPs and bytes of those launches (products count
+ * 2 * M * N * K, the full product even where only a triangle is computed).
+ * Returns the number of rows written, or a MUON_ERR_* code. */
+typedef struct {
+  const char* kernel;
+  int launches;
+  double ms;
+  double flops;
+  double bytes;
+} muon_profile_entry;
+MUON_API int muon_profile_begin(void);
+MUON_API int muon_profile_end(muon_profile_entry* out, int max_entries);
 
 /* Static text for a MUON_* return code or status bit set. */
 MUON_API const char* muon_status_string(int code);

@@ -21,7 +21,7 @@ __all__ = [
     "BF16", "FP16", "FP32", "STANDARD", "GRAM", "GRAM_STABILIZED", "QUINTIC", "CUBIC",
     "MuonError", "load_library", "library_path", "muon_step", "muon_ns_batched",
     "muon_workspace_size", "muon_workspace_min", "muon_ns_workspace_size", "muon_ns_flops",
-    "muon_status_string", "EXPORTED_SYMBOLS",
+    "muon_status_string", "muon_profile_begin", "muon_profile_end", "MuonStep", "EXPORTED_SYMBOLS",
 ]
 
 BF16, FP16, FP32 = 0, 1, 2
@@ -32,7 +32,7 @@ QUINTIC = (3.4445, -4.7750, 2.0315)
 CUBIC = (1.5, -0.5, 0.0)
 EXPORTED_SYMBOLS = (
     "muon_workspace_size", "muon_workspace_min", "muon_step", "muon_ns_workspace_size",
-    "muon_ns_batched", "muon_ns_flops", "muon_status_string",
+    "muon_ns_batched", "muon_ns_flops", "muon_status_string", "muon_profile_begin", "muon_profile_end",
 )
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -59,6 +59,11 @@ class _Group(ctypes.Structure):
 class _HParams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("momentum", ctypes.c_float), ("weight_decay", ctypes.c_float),
                 ("scale_coef", ctypes.c_float), ("nesterov", ctypes.c_int), ("ns", _NSParams)]
+
+
+class _ProfEntry(ctypes.Structure):
+    _fields_ = [("kernel", ctypes.c_char_p), ("launches", ctypes.c_int), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 def library_path() -> str:
@@ -89,6 +94,10 @@ def load_library() -> ctypes.CDLL:
     lib.muon_ns_batched.restype = ctypes.c_int
     lib.muon_ns_flops.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_NSParams)]
     lib.muon_ns_flops.restype = ctypes.c_double
+    lib.muon_profile_begin.argtypes = []
+    lib.muon_profile_begin.restype = ctypes.c_int
+    lib.muon_profile_end.argtypes = [ctypes.POINTER(_ProfEntry), ctypes.c_int]
+    lib.muon_profile_end.restype = ctypes.c_int
     lib.muon_status_string.argtypes = [ctypes.c_int]
     lib.muon_status_string.restype = ctypes.c_char_p
     _LIB = lib
@@ -278,3 +287,52 @@ def muon_ns_batched(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5, mode="s
                              ctypes.c_void_p(status.data_ptr() if status is not None else 0),
                              ctypes.c_void_p(_stream_handle(stream)))
     _raise(rc, "muon_ns_batched")
+
+
+def muon_profile_begin() -> None:
+    """Start bracketing every library launch with CUDA events (tracing aid)."""
+    _raise(load_library().muon_profile_begin(), "muon_profile_begin")
+
+
+def muon_profile_end() -> list[dict]:
+    """Stop profiling; per kernel kind: launches, device ms, algorithmic FLOPs and bytes."""
+    rows = (_ProfEntry * 16)()
+    n = load_library().muon_profile_end(rows, 16)
+    if n < 0:
+        _raise(n, "muon_profile_end")
+    return [dict(kernel=r.kernel.decode(), launches=r.launches, ms=r.ms, flops=r.flops, bytes=r.bytes)
+            for r in rows[:n]]
+
+
+class MuonStep:
+    """A prepared Muon step over a fixed set of tensors.
+
+    Builds the C structs (groups, hyper-parameters) and the workspace once, so
+    each call is a single C-ABI call with no per-step marshalling.  The tensors
+    must stay alive and keep their storage for the object's lifetime.
+    """
+
+    def __init__(self, params, grads, moms, *, workspace_bytes: int | None = None, **hp):
+        self._lib = load_library()
+        a = dict(_STEP_DEFAULTS, **hp)
+        self.hp = a
+        self._groups, self._ng, self._h, self._keep, self.order = _step_args(params, grads, moms, **a)
+        full = int(self._lib.muon_workspace_size(self._groups, self._ng, ctypes.byref(self._h)))
+        lo = int(self._lib.muon_workspace_min(self._groups, self._ng, ctypes.byref(self._h)))
+        if full == 0:
+            raise MuonError("invalid arguments (workspace query returned 0)")
+        size = full if workspace_bytes is None else max(lo, min(full, int(workspace_bytes)))
+        self.workspace = torch.empty(size, dtype=torch.uint8, device=params[0].device)
+        self.status = torch.zeros(len(self.order), dtype=torch.int32, device=params[0].device)
+        self.count = len(self.order)
+
+    def __call__(self, stream=None) -> None:
+        rc = self._lib.muon_step(self._groups, self._ng, ctypes.byref(self._h),
+                                 ctypes.c_void_p(self.workspace.data_ptr()), ctypes.c_size_t(self.workspace.numel()),
+                                 ctypes.c_void_p(self.status.data_ptr()), ctypes.c_void_p(_stream_handle(stream)))
+        _raise(rc, "muon_step")
+
+    def status_in_param_order(self) -> torch.Tensor:
+        out = torch.empty_like(self.status)
+        out[torch.tensor(self.order, device=out.device)] = self.status
+        return out

@@ -14,6 +14,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <mutex>
 #include <vector>
 
 #include "../../include/muon.h"
@@ -27,6 +28,48 @@ namespace {
 constexpr size_t kAlign = 256;
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int round8(int v) { return (v + 7) / 8 * 8; }
+
+// ------------------------------------------------------------------ profiler
+enum ProfKind { kProfPack, kProfNorm, kProfConvert, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfKinds };
+const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "scale_convert_kernel",
+                                            "gemm_kernel[symmetric]", "gemm_kernel", "gemm_simt_kernel",
+                                            "unpack_kernel"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+struct Profiler {
+  bool on = false;
+  std::vector<ProfRec> recs;
+  std::mutex mu;
+};
+Profiler& profiler() {
+  static Profiler p;
+  return p;
+}
+// Brackets one launch with events on its stream while profiling is on.
+struct ProfScope {
+  ProfRec rec{};
+  bool active = false;
+  cudaStream_t s;
+  ProfScope(int kind, double flops, double bytes, cudaStream_t st) : s(st) {
+    Profiler& P = profiler();
+    if (!P.on) return;
+    rec.kind = kind; rec.flops = flops; rec.bytes = bytes;
+    if (cudaEventCreate(&rec.a) != cudaSuccess) return;
+    if (cudaEventCreate(&rec.b) != cudaSuccess) { cudaEventDestroy(rec.a); return; }
+    cudaEventRecord(rec.a, s);
+    active = true;
+  }
+  ~ProfScope() {
+    if (!active) return;
+    cudaEventRecord(rec.b, s);
+    Profiler& P = profiler();
+    std::lock_guard<std::mutex> g(P.mu);
+    P.recs.push_back(rec);
+  }
+};
 
 struct Seg {          // `count` matrices of one caller group, starting at index `first`
   int group, first, count;
@@ -137,6 +180,12 @@ struct Ctx {
 
 int gemm(const Ctx& c, GemmDesc g) {
   g.err = c.err;
+  const double flops = 2.0 * g.M * g.N * (double)g.K * g.batch;
+  const int es = dtype_size(g.in_dtype);
+  const double bytes = ((double)g.M * g.K * es + (double)g.N * g.K * es + (double)g.M * g.N * dtype_size(g.d_dtype) +
+                        (g.C ? (double)g.M * g.N * dtype_size(g.c_dtype) : 0.0)) * g.batch;
+  const int kind = c.compute == MUON_FP32 ? kProfGemmSimt : (g.symmetric ? kProfSyrkTc : kProfGemmTc);
+  ProfScope ps(kind, flops, bytes, c.s);
   return c.compute == MUON_FP32 ? gemm_simt(g, c.s) : gemm_tc(g, c.s);
 }
 
@@ -148,18 +197,38 @@ GemmDesc desc(int M, int N, int K, int batch) {
   return g;
 }
 
-// Runs the Newton-Schulz chain on `chunk` packed matrices; returns the index of
-// the X buffer that holds the result through *out_x.
-int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, int* out_x) {
+// Runs the Newton-Schulz chain on `chunk` packed matrices (raw U in X[0], in
+// bf16 for the tensor-core path, fp32 for the SIMT path).  Returns the index
+// of the X buffer that holds the result and the result's dtype.
+//
+// 16-bit chains: the standard form stores X, A, B in compute_dtype; the Gram
+// forms store every matrix of the chain (R, Q, Q_acc, X0, restart X) in
+// gram_dtype, so that no product mixes operand types.  A bf16 chain applies
+// the normalisation f = 1/(||U||+eps) inside the first products' epilogues;
+// an fp16 chain first writes X0 = f U in fp16 (fp16's range cannot hold an
+// arbitrary raw gradient).
+int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, int* out_x,
+              int* out_dtype) {
   const int n = L.n, m = L.m, K = ns->iters;
-  const int xdt = c.compute;                                            // X storage
-  const int gdt = c.compute == MUON_FP32 ? MUON_FP32 : ns->gram_dtype;  // Gram storage
+  const int cdt = c.compute == MUON_FP32 ? MUON_FP32
+                                         : (ns->mode == MUON_NS_STANDARD ? ns->compute_dtype : ns->gram_dtype);
+  const int xdt = cdt;  // X storage
+  const int gdt = cdt;  // Gram-sized storage
   int rc;
+  int start = 0;
+  bool raw = true;
+  if (cdt == MUON_FP16) {
+    ProfScope ps(kProfConvert, 0.0, (double)chunk * B.x_bs * 4, c.s);
+    launch_scale_convert(B.X[0], B.X[1], B.inv, B.x_bs, chunk, c.s);
+    start = 1;
+    raw = false;
+  }
+  *out_dtype = xdt;
   if (ns->mode == MUON_NS_STANDARD) {
-    int cur = 0;
+    int cur = start;
     for (int k = 0; k < K; ++k) {
       const float a = ns->coeffs[3 * k], bb = ns->coeffs[3 * k + 1], cc = ns->coeffs[3 * k + 2];
-      const bool first = k == 0;
+      const bool first = k == 0 && raw;
       // A = f^2 X X^T  (f = 1/(||U||+eps) on the first iteration)
       GemmDesc g = desc(n, n, m, chunk);
       g.A = B.X[cur]; g.lda = L.ld_m; g.a_bs = B.x_bs;
@@ -203,8 +272,8 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
 
   // ---------------------------------------------------------------- Gram forms
   const bool stabilized = ns->mode == MUON_NS_GRAM_STABILIZED;
-  int x0 = 0;              // X buffer holding the matrix the Gram iteration applies to
-  bool x0_raw = true;      // still the unnormalised packed U (scale by inv on use)
+  int x0 = start;          // X buffer holding the matrix the Gram iteration applies to
+  bool x0_raw = raw;       // still the unnormalised packed U (scale by inv on use)
   void* R = B.S[0];
   void* T = B.S[1];
   void* Qbuf[3] = {B.S[2], B.S[3], B.S[4]};
@@ -237,7 +306,7 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
     return gemm(c, g);
   };
 
-  if ((rc = gram_of_x(true))) return rc;
+  if ((rc = gram_of_x(x0_raw))) return rc;
   for (int k = 1; k <= K; ++k) {
     const float a = ns->coeffs[3 * (k - 1)], bb = ns->coeffs[3 * (k - 1) + 1], cc = ns->coeffs[3 * (k - 1) + 2];
     const bool last = k == K;
@@ -273,10 +342,15 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
       if ((rc = gram_of_x(false))) return rc;
       q_acc = -1;
     } else {
-      // R <- Q R Q  as T = Q R, R = T Q
+      // R <- Q R Q  as T = Q R, R = T Q.  The second product is symmetric in
+      // exact arithmetic and is formed on the upper triangle and mirrored:
+      // the next Q takes R R^T (SYRK form), which equals R R only for an
+      // exactly symmetric R; a rounding-level antisymmetric part of R would
+      // otherwise enter Q through R R^T - R R and grow with every iteration.
       sq(g, Qbuf[qi], R, 0, T, gdt);
       if ((rc = gemm(c, g))) return rc;
       sq(g, T, Qbuf[qi], 0, R, gdt);
+      g.symmetric = 1;
       if ((rc = gemm(c, g))) return rc;
     }
   }
@@ -330,7 +404,7 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
         seg_i = si;
         seg_off = so;
       }
-      const int xdt = ns->compute_dtype;
+      const int pack_dt = ns->compute_dtype == MUON_FP32 ? MUON_FP32 : MUON_BF16;
       for (const Piece& pc : pieces) {
         const SrcView& v = views[pc.group];
         SegmentPtrs ptrs;
@@ -341,19 +415,24 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
         }
         PackArgs a{};
         a.rows = v.rows; a.cols = v.cols; a.count = pc.count;
-        a.src_dtype = v.src_dtype; a.x_dtype = xdt;
+        a.src_dtype = v.src_dtype; a.x_dtype = pack_dt;
         a.momentum_mode = update ? 1 : 0; a.mu = mu; a.nesterov = nesterov;
         a.x = reinterpret_cast<char*>(B.X[0]) + (size_t)pc.slot * B.x_bs * L.x_es;
         a.ld_x = L.ld_m; a.x_batch_stride = B.x_bs;
         a.partials = B.partials + (size_t)pc.slot * L.tiles;
         a.partial_stride = L.tiles;
+        const double elems = (double)v.rows * v.cols * pc.count;
+        ProfScope ps(kProfPack, 0.0, elems * (dtype_size(v.src_dtype) + L.x_es + (update ? 8 : 0)), s);
         launch_pack(a, ptrs, s);
       }
-      launch_norm(B.partials, L.tiles, L.tiles, chunk, ns->eps, B.inv, s);
+      {
+        ProfScope ps(kProfNorm, 0.0, (double)chunk * L.tiles * 4 + chunk * 4.0, s);
+        launch_norm(B.partials, L.tiles, L.tiles, chunk, ns->eps, B.inv, s);
+      }
       if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
       Ctx ctx{ns->compute_dtype, s, B.err};
-      int xi = 0;
-      if (run_chain(ctx, L, B, chunk, ns, &xi) != 0) return MUON_ERR_CUDA;
+      int xi = 0, out_dt = pack_dt;
+      if (run_chain(ctx, L, B, chunk, ns, &xi, &out_dt) != 0) return MUON_ERR_CUDA;
       for (const Piece& pc : pieces) {
         const SrcView& v = views[pc.group];
         SegmentPtrs ptrs;
@@ -364,7 +443,7 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
         }
         UnpackArgs u{};
         u.rows = v.rows; u.cols = v.cols; u.count = pc.count;
-        u.dst_dtype = v.dst_dtype; u.x_dtype = xdt;
+        u.dst_dtype = v.dst_dtype; u.x_dtype = out_dt;
         u.update_mode = update ? 1 : 0;
         u.decay = 1.f - lr * wd;
         u.step = lr * scale_coef * std::sqrt((float)std::max(v.rows, v.cols));
@@ -372,6 +451,8 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
         u.ld_x = L.ld_m; u.x_batch_stride = B.x_bs;
         u.status = status ? status + first_index[pc.group] + pc.first : nullptr;
         u.chunk_err = B.err;
+        const double elems = (double)v.rows * v.cols * pc.count;
+        ProfScope ps(kProfUnpack, 0.0, elems * (L.x_es + dtype_size(v.dst_dtype) * (update ? 2 : 1)), s);
         launch_unpack(u, ptrs, s);
       }
       if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
@@ -513,6 +594,41 @@ int muon_ns_batched(void* const* X, int count, int rows, int cols, int dtype, co
 double muon_ns_flops(int rows, int cols, const muon_ns_params* ns) {
   if (rows <= 0 || cols <= 0 || !ns_params_ok(ns)) return 0.0;
   return flops_of(rows, cols, ns);
+}
+
+int muon_profile_begin(void) {
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> g(P.mu);
+  for (auto& r : P.recs) { cudaEventDestroy(r.a); cudaEventDestroy(r.b); }
+  P.recs.clear();
+  P.on = true;
+  return MUON_OK;
+}
+
+int muon_profile_end(muon_profile_entry* out, int max_entries) {
+  Profiler& P = profiler();
+  std::lock_guard<std::mutex> g(P.mu);
+  P.on = false;
+  muon_profile_entry acc[kProfKinds];
+  for (int k = 0; k < kProfKinds; ++k) acc[k] = muon_profile_entry{kProfNames[k], 0, 0.0, 0.0, 0.0};
+  int rc = MUON_OK;
+  for (auto& r : P.recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) rc = MUON_ERR_CUDA;
+    acc[r.kind].launches += 1;
+    acc[r.kind].ms += ms;
+    acc[r.kind].flops += r.flops;
+    acc[r.kind].bytes += r.bytes;
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  P.recs.clear();
+  if (rc != MUON_OK) return rc;
+  if (!out && max_entries > 0) return MUON_ERR_INVALID;
+  int n = 0;
+  for (int k = 0; k < kProfKinds && n < max_entries; ++k)
+    if (acc[k].launches) out[n++] = acc[k];
+  return n;
 }
 
 const char* muon_status_string(int code) {

@@ -261,6 +261,27 @@ unpack_kernel(const UnpackArgs a, const __grid_constant__ SegmentPtrs p) {
 }
 
 // ----------------------------------------------------------------------------
+// normalise + convert: dst[b] = inv[b] * src[b] (bf16 -> fp16), 8 elements per
+// thread with 128-bit loads and stores; per_matrix is a multiple of 8
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+scale_convert_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, const float* __restrict__ inv,
+                     long long per_matrix, long long total) {
+  const long long n8 = total / 8;
+  for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8; v += (long long)gridDim.x * blockDim.x) {
+    const long long i = v * 8;
+    const float f = inv[i / per_matrix];
+    const uint4 q = reinterpret_cast<const uint4*>(src)[v];
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&q);
+    uint4 o;
+    __half* h = reinterpret_cast<__half*>(&o);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) h[k] = __float2half_rn(f * __bfloat162float(e[k]));
+    reinterpret_cast<uint4*>(dst)[v] = o;
+  }
+}
+
+// ----------------------------------------------------------------------------
 // dtype conversion of a flat array (rare Gram-mode corner cases)
 // ----------------------------------------------------------------------------
 __global__ void convert_kernel(const void* src, int sdt, void* dst, int ddt, long long n) {
@@ -336,6 +357,17 @@ void launch_unpack(const UnpackArgs& a, const SegmentPtrs& p, cudaStream_t s) {
     case kFP16: unpack_dispatch1<__half>(a, p, s); break;
     default: unpack_dispatch1<float>(a, p, s); break;
   }
+}
+
+void launch_scale_convert(const void* src, void* dst, const float* inv, long long per_matrix, int count,
+                          cudaStream_t s) {
+  const long long total = per_matrix * count;
+  if (total <= 0) return;
+  long long blocks = (total / 8 + 255) / 256;
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  scale_convert_kernel<<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(src),
+                                                   reinterpret_cast<__half*>(dst), inv, per_matrix, total);
 }
 
 void launch_convert(const void* src, int sdt, void* dst, int ddt, long long n, cudaStream_t s) {

@@ -17,6 +17,8 @@ gemm_simt_kernel(const GemmDesc g) {
   __shared__ __align__(16) float Bs[kSK][kSB + 4];
   const int b = blockIdx.z;
   const int i0 = blockIdx.y * kSB, j0 = blockIdx.x * kSB;
+  // symmetric results: blocks below the diagonal are mirrors of blocks above it
+  if (g.symmetric && blockIdx.x < blockIdx.y) return;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const T* A = reinterpret_cast<const T*>(g.A) + (long long)b * g.a_bs;
   const T* B = reinterpret_cast<const T*>(g.B) + (long long)b * g.b_bs;
@@ -74,6 +76,13 @@ gemm_simt_kernel(const GemmDesc g) {
       if (C) v += g.c_in * load_any(C, (long long)gi * g.ldc + gj, g.c_dtype);
       v *= f;
       if (gi == gj) v += g.c_eye;
+      if (g.symmetric) {
+        // upper triangle stored twice (direct and mirrored): exactly symmetric
+        if (gj < gi) continue;
+        store_any(D, (long long)gi * g.ldd + gj, g.d_dtype, v);
+        if (gj != gi) store_any(D, (long long)gj * g.ldd + gi, g.d_dtype, v);
+        continue;
+      }
       store_any(D, (long long)gi * g.ldd + gj, g.d_dtype, v);
     }
   }

@@ -24,266 +24,13 @@
 // Every mbarrier wait is bounded (global-timer deadline plus a CTA-wide abort
 // flag); on expiry the CTA drains its in-flight copies and MMAs, frees TMEM,
 // raises the timeout bit in the caller's error word and returns.
-#include <cuda.h>
 #include <stdio.h>
 #include <stdlib.h>
 
-#include "common.cuh"
-#include "internal.h"
+#include "tc_common.cuh"
 
 namespace muon {
 namespace tc {
-
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;                   // 64 x 2 B = one 128-byte swizzle row
-constexpr int UMMA_K = 16;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;     // 16 KB
-constexpr int B_BYTES = BN * BK * 2;     // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
-constexpr int TMEM_COLS = 2 * BN;        // two fp32 accumulators
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr int GROUP_M = 8;               // tile raster grouping for L2 reuse
-
-struct Params {
-  int M, N, K, batch;
-  int tiles_m, tiles_n, tiles_per_batch, total_tiles;
-  int symmetric;
-  void* D; int ldd; long long d_bs; int d_dtype;
-  const void* C; int ldc; long long c_bs; int c_dtype;
-  float c_acc, c_in, c_eye;
-  const float* scale; int scale_pow;
-  int* err;
-  long long timeout_ns;
-};
-
-// ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t global_timer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false when the deadline passed or another role aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          long long timeout_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer();
-  for (uint32_t it = 1; it < (1u << 30); ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0) {
-      if (*abort_flag) return false;
-      if ((long long)(global_timer() - t0) > timeout_ns) {
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-  *abort_flag = 1;
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
-                                            int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
-  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-  return d;
-}
-
-// Instruction descriptor for kind::f16: fp32 D, A/B of one 16-bit type,
-// A K-major, B K-major or MN-major, M = 128, N = 256.
-__host__ __device__ constexpr uint32_t make_idesc(int in_fmt /*0 f16, 1 bf16*/, int b_mn) {
-  return (1u << 4) | ((uint32_t)in_fmt << 7) | ((uint32_t)in_fmt << 10) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-}
-
-// ------------------------------------------------------------------ tile order
-struct Tile { int b, tm, tn; };
-
-__device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
-  Tile r;
-  r.b = t / p.tiles_per_batch;
-  int q = t - r.b * p.tiles_per_batch;
-  if (p.symmetric) {
-    // upper-triangle tiles in 128-block units: row tm keeps tn >= tm / 2
-    int tm = 0;
-    for (; tm < p.tiles_m; ++tm) {
-      const int cnt = p.tiles_n - tm / 2;
-      if (q < cnt) break;
-      q -= cnt;
-    }
-    r.tm = tm;
-    r.tn = tm / 2 + q;
-  } else {
-    const int per_group = GROUP_M * p.tiles_n;
-    const int g = q / per_group;
-    const int first = g * GROUP_M;
-    const int gsz = min(p.tiles_m - first, GROUP_M);
-    const int w = q - g * per_group;
-    r.tm = first + w % gsz;
-    r.tn = w / gsz;
-  }
-  return r;
-}
-
-// ------------------------------------------------------------------ epilogue
-__device__ __forceinline__ void store_row32(void* D, int dt, long long off, const float* v) {
-  uint4 q[4];
-  if (dt == kBF16) {
-    __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(q);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) e[i] = __float2bfloat16_rn(v[i]);
-    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(D) + off);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = q[i];
-  } else {
-    __half* e = reinterpret_cast<__half*>(q);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) e[i] = __float2half_rn(v[i]);
-    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(D) + off);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = q[i];
-  }
-}
-
-__device__ __forceinline__ void load_row32(const void* C, int dt, long long off, float* v) {
-  uint4 q[4];
-  const uint4* s = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(C) + off * 2);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) q[i] = s[i];
-  if (dt == kBF16) {
-    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(q);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(e[i]);
-  } else {
-    const __half* e = reinterpret_cast<const __half*>(q);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __half2float(e[i]);
-  }
-}
-
-__device__ __forceinline__ void epilogue_chunk(const Params& p, const Tile& t, int row_in_tile, int chunk,
-                                               const uint32_t (&acc)[32], float f) {
-  const int gi = t.tm * BM + row_in_tile;
-  const int gj0 = t.tn * BN + chunk * 32;
-  bool mirror = false;
-  if (p.symmetric) {
-    const int bj = t.tn * 2 + (chunk >> 2);  // 128-column block of this chunk
-    if (bj < t.tm) return;                   // lower block: its mirror is stored elsewhere
-    mirror = bj > t.tm;
-  }
-  if (gi >= p.M || gj0 >= p.N) return;
-  const bool full = (gj0 + 32 <= p.N);
-  float v[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = p.c_acc * __uint_as_float(acc[j]);
-  if (p.C != nullptr) {
-    const char* cb = reinterpret_cast<const char*>(p.C) + (long long)t.b * p.c_bs * 2;
-    const long long off = (long long)gi * p.ldc + gj0;
-    if (full) {
-      float c[32];
-      load_row32(cb, p.c_dtype, off, c);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] += p.c_in * c[j];
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (gj0 + j < p.N) v[j] += p.c_in * load_any(cb, off + j, p.c_dtype);
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    v[j] *= f;
-    if (gj0 + j == gi) v[j] += p.c_eye;
-  }
-
-  char* db = reinterpret_cast<char*>(p.D) + (long long)t.b * p.d_bs * 2;
-  {
-    const long long off = (long long)gi * p.ldd + gj0;
-    if (full) {
-      store_row32(db, p.d_dtype, off, v);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (gj0 + j < p.N) store_any(db, off + j, p.d_dtype, v[j]);
-    }
-  }
-  if (mirror) {
-    // D[gj][gi]: for each j the warp's 32 rows form 32 consecutive columns.
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (gj0 + j < p.N) store_any(db, (long long)(gj0 + j) * p.ldd + gi, p.d_dtype, v[j]);
-  }
-}
 
 // ------------------------------------------------------------------ kernel
 template <bool B_MN, int IN_FMT>
@@ -292,7 +39,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
             const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint16_t* staging = reinterpret_cast<uint16_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + STAGING_BYTES);
   uint64_t* full_bar = bars;                    // [STAGES]
   uint64_t* empty_bar = bars + STAGES;          // [STAGES]
   uint64_t* tfull_bar = bars + 2 * STAGES;      // [2]
@@ -310,7 +58,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull_bar[a]), 1);
-      mbar_init(smem_u32(&tempty_bar[a]), 128);
+      mbar_init(smem_u32(&tempty_bar[a]), 32 * NUM_EPI_WARPS);
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
@@ -408,8 +156,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int row_in_tile = q * 32 + lane;
+    const int q = warp & 3;                      // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;            // which 4 of the 8 column chunks
+    uint16_t* stage = staging + (warp - 2) * (STAGE_BYTES_PER_WARP / 2);
     int it = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
       const Tile tl = decode_tile(p, t);
@@ -422,15 +171,28 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
       tc_fence_after();
       const float f = matrix_scale(p.scale, p.scale_pow, tl.b);
       const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      const int gi = tl.tm * BM + q * 32 + lane;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = half * 4 + cc;
+        const int gj0 = tl.tn * BN + c * 32;
+        // C row segment first, so its latency overlaps the TMEM read
+        uint4 creg[4];
+        bool c_ready = false;
+        if (p.C != nullptr && gi < p.M && gj0 + 32 <= p.N) {
+          const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.C) +
+                                                            ((long long)tl.b * p.c_bs + (long long)gi * p.ldc + gj0) * 2);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) creg[i] = src[i];
+          c_ready = true;
+        }
         uint32_t r[32];
         tmem_ld32(tbase + (uint32_t)(c * 32), r);
-        if (c == BN / 32 - 1) {
+        if (cc == 3) {
           tc_fence_before();
           mbar_arrive(smem_u32(&tempty_bar[acc]));
         }
-        epilogue_chunk(p, tl, row_in_tile, c, r, f);
+        epilogue_chunk(p, tl, q, lane, c, r, creg, c_ready, f, stage);
       }
     }
   }
@@ -464,7 +226,7 @@ static EncodeTiledFn get_encode() {
 }
 
 // 3-D tiled map over a batch of row-major matrices: dims (inner, outer, batch).
-static bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer,
+bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer,
                        long long batch, long long ld_elems, long long bs_elems, int box_inner, int box_outer) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
@@ -521,6 +283,15 @@ int gemm_tc(const GemmDesc& g, cudaStream_t s) {
   p.scale = g.scale; p.scale_pow = g.scale_pow;
   p.err = g.err;
   p.timeout_ns = wait_timeout_ns();
+
+  // 256-row products go to the paired-CTA kernel (a third less operand
+  // traffic per MMA); MUON_GEMM_PAIR=0 keeps every product on the 1-CTA one.
+  static int use_pair = -1;
+  if (use_pair < 0) {
+    const char* e = getenv("MUON_GEMM_PAIR");
+    use_pair = (e && e[0] == '0') ? 0 : 1;
+  }
+  if (use_pair && g.M >= 256) return gemm_tc_pair(g, p, s);
 
   CUtensorMap ma, mb;
   if (!encode_map(&ma, g.in_dtype, g.A, g.K, g.M, g.batch, g.lda, g.a_bs, BK, BM)) return (int)cudaErrorInvalidValue;

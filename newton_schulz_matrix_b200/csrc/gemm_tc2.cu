@@ -1,0 +1,333 @@
+// Paired-CTA (cta_group::2) variant of the tensor-core product kernel.
+//
+// Same computation and epilogue as the 1-CTA kernel (gemm_tc.cu), on 256 x 256
+// output tiles owned by a cluster of two CTAs on two SMs:
+//   - each CTA loads its own 128 rows of A and its own 128 of the tile's 256
+//     columns of B (plain TMA loads in the cta_group::2 form, which report
+//     completion to the leader CTA's barrier; no multicast), so a CTA moves
+//     32 KB per 64-deep k-step for 128 x 256 x 64 MACs instead of 48 KB;
+//   - the leader CTA issues one M=256, N=256, K=16 tcgen05.mma per k16 that
+//     reads both CTAs' shared memory and writes both CTAs' TMEM (128 lanes
+//     each), and releases each stage in both CTAs with a multicast commit;
+//   - each CTA drains its own 128 x 256 accumulator (two TMEM buffers) with
+//     the shared epilogue; both CTAs' epilogue warps hand the buffer back to
+//     the leader's MMA issuer through a remote mbarrier arrive.
+// Waits are bounded as in the 1-CTA kernel.
+#include <stdio.h>
+
+#include "tc_common.cuh"
+
+namespace muon {
+namespace tc {
+namespace pairk {
+
+constexpr int STAGES2 = 6;
+constexpr int A_BYTES2 = BM * BK * 2;   // this CTA's 128 rows of A: 16 KB
+constexpr int B_BYTES2 = 128 * BK * 2;  // this CTA's 128 columns of B: 16 KB
+constexpr int STAGE_BYTES2 = A_BYTES2 + B_BYTES2;
+constexpr int SMEM_BYTES2 = STAGES2 * STAGE_BYTES2 + STAGING_BYTES + 1024 + 256;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive (once MMAs issued so far retire) on the barrier at this offset in
+// every CTA of `mask`.
+__device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void remote_arrive(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+struct PairTile { int b, TM, TN; };
+
+__device__ __forceinline__ PairTile decode_pair(const Params& p, int t) {
+  PairTile r;
+  r.b = t / p.tiles_per_batch;
+  int q = t - r.b * p.tiles_per_batch;
+  if (p.symmetric) {
+    int tm = 0;
+    for (; tm < p.tiles_m; ++tm) {
+      const int cnt = p.tiles_n - tm;
+      if (q < cnt) break;
+      q -= cnt;
+    }
+    r.TM = tm;
+    r.TN = tm + q;
+  } else {
+    const int per_group = GROUP_M * p.tiles_n;
+    const int g = q / per_group;
+    const int first = g * GROUP_M;
+    const int gsz = min(p.tiles_m - first, GROUP_M);
+    const int w = q - g * per_group;
+    r.TM = first + w % gsz;
+    r.TN = w / gsz;
+  }
+  return r;
+}
+
+template <bool B_MN, int IN_FMT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                 const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint16_t* staging = reinterpret_cast<uint16_t*>(smem + STAGES2 * STAGE_BYTES2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES2 * STAGE_BYTES2 + STAGING_BYTES);
+  uint64_t* full_bar = bars;                      // [STAGES2]   (used in the leader)
+  uint64_t* empty_bar = bars + STAGES2;           // [STAGES2]   (both CTAs)
+  uint64_t* tfull_bar = bars + 2 * STAGES2;       // [2]         (both CTAs)
+  uint64_t* tempty_bar = bars + 2 * STAGES2 + 2;  // [2]         (used in the leader)
+  uint64_t* drain_bar = bars + 2 * STAGES2 + 4;   // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES2 + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0 = leader, 1 = peer
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&tfull_bar[a]), 1);
+      mbar_init(smem_u32(&tempty_bar[a]), 2 * NUM_EPI_WARPS);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int num_kb = (p.K + BK - 1) / BK;
+  const uint32_t leader_full = mapa(smem_u32(full_bar), 0);
+  const uint32_t leader_tempty = mapa(smem_u32(tempty_bar), 0);
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producers (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < p.total_tiles && ok; t += npairs) {
+        const PairTile tl = decode_pair(p, t);
+        const int row0 = tl.TM * 256 + (int)rank * 128;   // this CTA's rows of A
+        const int col0 = tl.TN * 256 + (int)rank * 128;   // this CTA's columns of B
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+          if (leader) mbar_expect_tx(smem_u32(&full_bar[stage]), 2 * STAGE_BYTES2);
+          const uint32_t fb = leader_full + stage * 8;
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES2);
+          const uint32_t sb = sa + A_BYTES2;
+          tma_load_3d_pair(sa, &tmap_a, fb, kb * BK, row0, tl.b);
+          if (B_MN) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) tma_load_3d_pair(sb + q * (BK * 128), &tmap_b, fb, col0 + q * 64, kb * BK, tl.b);
+          } else {
+            tma_load_3d_pair(sb, &tmap_b, fb, kb * BK, col0, tl.b);
+          }
+          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // no drain needed here: the leader's MMAs consume every issued stage,
+      // and the final cluster barrier keeps this CTA resident until then
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer (leader only)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = make_idesc(IN_FMT, B_MN ? 1 : 0, 256);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = pair; t < p.total_tiles && ok; t += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(smem_u32(&tempty_bar[acc]), aph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES2);
+          const uint32_t sb = sa + A_BYTES2;
+#pragma unroll
+          for (int k = 0; k < BK / UMMA_K; ++k) {
+            const uint64_t ad = smem_desc(sa + k * (UMMA_K * 2), 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc(sb + k * (UMMA_K * 128), BK * 128, 1024)
+                                     : smem_desc(sb + k * (UMMA_K * 2), 16, 1024);
+            mma_pair(d_tmem, ad, bd, idesc, (kb | k) != 0);
+          }
+          commit_pair(smem_u32(&empty_bar[stage]), 0x3);  // stage free in both CTAs
+          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        commit_pair(smem_u32(&tfull_bar[acc]), 0x3);      // accumulator ready in both CTAs
+      }
+      commit_pair(smem_u32(drain_bar), 0x1);
+      volatile int never = 0;
+      mbar_wait(smem_u32(drain_bar), 0, &never, p.timeout_ns);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    uint16_t* stage = staging + (warp - 2) * (STAGE_BYTES_PER_WARP / 2);
+    int it = 0;
+    for (int t = pair; t < p.total_tiles; t += npairs, ++it) {
+      const PairTile pt = decode_pair(p, t);
+      const Tile tl{pt.b, pt.TM * 2 + (int)rank, pt.TN};
+      const int acc = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(smem_u32(&tfull_bar[acc]), aph, abort_flag, p.timeout_ns);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const float f = matrix_scale(p.scale, p.scale_pow, tl.b);
+      const uint32_t tbase = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(q * 32) << 16);
+      const int gi = tl.tm * BM + q * 32 + lane;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = half * 4 + cc;
+        const int gj0 = tl.tn * BN + c * 32;
+        uint4 creg[4];
+        bool c_ready = false;
+        if (p.C != nullptr && gi < p.M && gj0 + 32 <= p.N) {
+          const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.C) +
+                                                            ((long long)tl.b * p.c_bs + (long long)gi * p.ldc + gj0) * 2);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) creg[i] = src[i];
+          c_ready = true;
+        }
+        uint32_t r[32];
+        tmem_ld32(tbase + (uint32_t)(c * 32), r);
+        if (cc == 3) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) remote_arrive(leader_tempty + acc * 8);
+        }
+        epilogue_chunk(p, tl, q, lane, c, r, creg, c_ready, f, stage);
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the leader's MMAs into this CTA's TMEM are drained
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+  if (threadIdx.x == 0 && *abort_flag && p.err != nullptr) atomicOr(p.err, kStatusTimeout);
+}
+
+template <bool B_MN, int IN_FMT>
+static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+  static int max_pairs = 0;
+  auto kern = gemm_pair_kernel<B_MN, IN_FMT>;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES2;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (max_pairs == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES2);
+    if (e != cudaSuccess) return (int)e;
+    cfg.gridDim = dim3(2 * (num_sms() / 2));
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess || n <= 0) n = num_sms() / 2;
+    max_pairs = n;
+  }
+  const int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
+  cfg.gridDim = dim3(2 * pairs);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+  return (int)e;
+}
+
+}  // namespace pairk
+
+int gemm_tc_pair(const GemmDesc& g, Params p, cudaStream_t s) {
+  using namespace pairk;
+  // pair tiles: 256 rows x 256 columns
+  p.tiles_m = (g.M + 255) / 256;
+  p.tiles_n = (g.N + BN - 1) / BN;
+  if (g.symmetric) {
+    p.tiles_per_batch = p.tiles_m * (p.tiles_m + 1) / 2;  // M == N: tiles_m == tiles_n
+  } else {
+    p.tiles_per_batch = p.tiles_m * p.tiles_n;
+  }
+  const long long total = (long long)p.tiles_per_batch * g.batch;
+  if (total > 0x7fffffffLL) return (int)cudaErrorInvalidValue;
+  p.total_tiles = (int)total;
+  CUtensorMap ma, mb;
+  if (!encode_map(&ma, g.in_dtype, g.A, g.K, g.M, g.batch, g.lda, g.a_bs, BK, BM)) return (int)cudaErrorInvalidValue;
+  const bool bmn = !g.b_kmajor;
+  if (bmn) {
+    if (!encode_map(&mb, g.in_dtype, g.B, g.N, g.K, g.batch, g.ldb, g.b_bs, 64, BK)) return (int)cudaErrorInvalidValue;
+  } else {
+    if (!encode_map(&mb, g.in_dtype, g.B, g.K, g.N, g.batch, g.ldb, g.b_bs, BK, 128)) return (int)cudaErrorInvalidValue;
+  }
+  const int fmt = g.in_dtype == kBF16 ? 1 : 0;
+  if (bmn) return fmt ? launch<true, 1>(ma, mb, p, s) : launch<true, 0>(ma, mb, p, s);
+  return fmt ? launch<false, 1>(ma, mb, p, s) : launch<false, 0>(ma, mb, p, s);
+}
+
+}  // namespace tc
+}  // namespace muon

@@ -52,7 +52,10 @@ struct UnpackArgs {
 };
 void launch_unpack(const UnpackArgs& a, const SegmentPtrs& p, cudaStream_t s);
 
-// Fill n x n identity-free helpers
+// dst[b] = inv[b] * src[b]: bf16 raw U -> fp16 X0 (per_matrix elements each,
+// a multiple of 8).
+void launch_scale_convert(const void* src, void* dst, const float* inv, long long per_matrix, int count,
+                          cudaStream_t s);
 void launch_convert(const void* src, int src_dtype, void* dst, int dst_dtype, long long n,
                     cudaStream_t s);
 

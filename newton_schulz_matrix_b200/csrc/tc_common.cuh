@@ -1,0 +1,311 @@
+// Device-side building blocks shared by the tcgen05 product kernels (1-CTA
+// and 2-CTA): constants, launch parameters, PTX wrappers for mbarriers, TMA,
+// tcgen05 MMA / TMEM, shared-memory descriptors, the tile order and the
+// fused polynomial epilogue.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace muon {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;                   // 64 x 2 B = one 128-byte swizzle row
+constexpr int UMMA_K = 16;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int B_BYTES = BN * BK * 2;     // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_EPI_WARPS = 8;         // two per TMEM lane quarter, 4 chunks of 32 columns each
+constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int TMEM_COLS = 2 * BN;        // two fp32 accumulators
+constexpr int STAGING_BYTES = NUM_EPI_WARPS * 32 * 40 * 2;  // mirrored-store staging tiles
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int GROUP_M = 8;               // tile raster grouping for L2 reuse
+
+struct Params {
+  int M, N, K, batch;
+  int tiles_m, tiles_n, tiles_per_batch, total_tiles;
+  int symmetric;
+  void* D; int ldd; long long d_bs; int d_dtype;
+  const void* C; int ldc; long long c_bs; int c_dtype;
+  float c_acc, c_in, c_eye;
+  const float* scale; int scale_pow;
+  int* err;
+  long long timeout_ns;
+};
+
+// ------------------------------------------------------------------ PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t global_timer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the deadline passed or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if ((long long)(global_timer() - t0) > timeout_ns) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor for kind::f16: fp32 D, A/B of one 16-bit type,
+// A K-major, B K-major or MN-major, M = 128, N = 256.
+__host__ __device__ constexpr uint32_t make_idesc(int in_fmt /*0 f16, 1 bf16*/, int b_mn, int m = BM) {
+  return (1u << 4) | ((uint32_t)in_fmt << 7) | ((uint32_t)in_fmt << 10) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ tile order
+struct Tile { int b, tm, tn; };
+
+__device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
+  Tile r;
+  r.b = t / p.tiles_per_batch;
+  int q = t - r.b * p.tiles_per_batch;
+  if (p.symmetric) {
+    // upper-triangle tiles in 128-block units: row tm keeps tn >= tm / 2
+    int tm = 0;
+    for (; tm < p.tiles_m; ++tm) {
+      const int cnt = p.tiles_n - tm / 2;
+      if (q < cnt) break;
+      q -= cnt;
+    }
+    r.tm = tm;
+    r.tn = tm / 2 + q;
+  } else {
+    const int per_group = GROUP_M * p.tiles_n;
+    const int g = q / per_group;
+    const int first = g * GROUP_M;
+    const int gsz = min(p.tiles_m - first, GROUP_M);
+    const int w = q - g * per_group;
+    r.tm = first + w % gsz;
+    r.tn = w / gsz;
+  }
+  return r;
+}
+
+// ------------------------------------------------------------------ epilogue
+__device__ __forceinline__ void store_row32(void* D, int dt, long long off, const float* v) {
+  uint4 q[4];
+  if (dt == kBF16) {
+    __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) e[i] = __float2bfloat16_rn(v[i]);
+    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(D) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = q[i];
+  } else {
+    __half* e = reinterpret_cast<__half*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) e[i] = __float2half_rn(v[i]);
+    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(D) + off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = q[i];
+  }
+}
+
+__device__ __forceinline__ void cvt_row32(const uint4 (&q)[4], int dt, float* v) {
+  if (dt == kBF16) {
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(e[i]);
+  } else {
+    const __half* e = reinterpret_cast<const __half*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __half2float(e[i]);
+  }
+}
+
+__device__ __forceinline__ uint16_t to_bits(float v, int dt) {
+  if (dt == kBF16) return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  return __half_as_ushort(__float2half_rn(v));
+}
+
+// Per-warp shared staging tile for the mirrored (transposed) store of one
+// 32 x 32 chunk: 32 rows of 40 halfwords (80-byte stride keeps the row-wise
+// 16-byte reads free of bank conflicts).
+constexpr int STAGE_LD = 40;
+constexpr int STAGE_BYTES_PER_WARP = 32 * STAGE_LD * 2;
+
+// One 32 x 32 chunk of the output: this warp's 32 tile rows (one per lane,
+// TMEM lane quarter q) times columns [gj0, gj0 + 32).  `creg` holds the C row
+// segment when `c_ready` (loaded before the TMEM read to hide its latency).
+__device__ __forceinline__ void epilogue_chunk(const Params& p, const Tile& t, int q, int lane, int chunk,
+                                               const uint32_t (&acc)[32], const uint4 (&creg)[4], bool c_ready,
+                                               float f, uint16_t* stage) {
+  const int gi_base = t.tm * BM + q * 32;
+  const int gi = gi_base + lane;
+  const int gj0 = t.tn * BN + chunk * 32;
+  // 0: plain store; 1: store + mirror; 2: diagonal block (upper half + mirror)
+  int kind = 0;
+  if (p.symmetric) {
+    const int bj = t.tn * 2 + (chunk >> 2);  // 128-column block of this chunk
+    if (bj < t.tm) return;                   // lower block: stored as the mirror of its transpose
+    kind = bj > t.tm ? 1 : 2;
+  }
+  if (gj0 >= p.N || gi_base >= p.M) return;  // warp-uniform
+  const bool full = gj0 + 32 <= p.N;
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = p.c_acc * __uint_as_float(acc[j]);
+  if (p.C != nullptr && gi < p.M) {
+    if (c_ready) {
+      float c[32];
+      cvt_row32(creg, p.c_dtype, c);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += p.c_in * c[j];
+    } else {
+      const char* cb = reinterpret_cast<const char*>(p.C) + (long long)t.b * p.c_bs * 2;
+      const long long off = (long long)gi * p.ldc + gj0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (gj0 + j < p.N) v[j] += p.c_in * load_any(cb, off + j, p.c_dtype);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    v[j] *= f;
+    if (gj0 + j == gi) v[j] += p.c_eye;
+  }
+
+  char* db = reinterpret_cast<char*>(p.D) + (long long)t.b * p.d_bs * 2;
+  // direct store of row gi (diagonal blocks: only columns >= gi)
+  if (gi < p.M) {
+    const long long off = (long long)gi * p.ldd + gj0;
+    if (full && (kind != 2 || gj0 >= gi)) {
+      store_row32(db, p.d_dtype, off, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (gj0 + j < p.N && (kind != 2 || gj0 + j >= gi)) store_any(db, off + j, p.d_dtype, v[j]);
+    }
+  }
+  if (kind == 0) return;
+  // mirrored store D[gj][gi] through the staging tile: lane l writes target row gj0 + l
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stage[j * STAGE_LD + lane] = to_bits(v[j], p.d_dtype);
+  __syncwarp();
+  const int row = gj0 + lane;
+  if (row < p.N) {
+    uint4 w[4];
+    const uint4* src = reinterpret_cast<const uint4*>(stage + lane * STAGE_LD);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w[i] = src[i];
+    uint16_t* drow = reinterpret_cast<uint16_t*>(db) + (long long)row * p.ldd + gi_base;
+    // valid columns: gi_base + k < M, and for diagonal blocks strictly below the diagonal (k < row - gi_base)
+    const int lim_m = p.M - gi_base;
+    const int lim = kind == 2 ? min(lim_m, row - gi_base) : lim_m;
+    if (lim >= 32) {
+      uint4* d = reinterpret_cast<uint4*>(drow);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) d[i] = w[i];
+    } else {
+      const uint16_t* e = reinterpret_cast<const uint16_t*>(w);
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        if (k < lim) drow[k] = e[k];
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side (gemm_tc.cu)
+// 3-D tiled tensor map over a batch of row-major matrices, 128-byte swizzle.
+bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer, long long batch,
+                long long ld_elems, long long bs_elems, int box_inner, int box_outer);
+// 2-CTA (cta_group::2) variant for 256-row tiles (gemm_tc2.cu).
+int gemm_tc_pair(const GemmDesc& g, Params p, cudaStream_t s);
+
+}  // namespace tc
+}  // namespace muon
