@@ -141,6 +141,30 @@ MUON_API size_t muon_ns_workspace_size(int count, int rows, int cols, const muon
 MUON_API int muon_ns_batched(void* const* X, int count, int rows, int cols, int dtype, const muon_ns_params* ns, void* ws,
                     size_t ws_bytes, int* status_per_matrix, void* stream);
 
+/* muon_ns_batched without a caller workspace, for callers that cannot
+ * allocate device memory when they orthogonalise: a host whose caching
+ * allocator already owns the GPU's memory (a raw cudaMalloc would fail or
+ * fragment its pool), a loop that forbids allocation after start-up, or a
+ * plugin that receives only input/output pointers.  The pages have no
+ * counterpart of this entry point; it is a library convenience.
+ *
+ * The workspace is a fixed array of MUON_NOALLOC_SCRATCH_BYTES inside the
+ * library, present on every GPU that loads the library until the process
+ * exits.  The call allocates and frees nothing.  A shape whose one-matrix
+ * workspace (muon_ns_workspace_size(1, rows, cols, ns)) exceeds the array is
+ * rejected with MUON_ERR_WORKSPACE; larger counts of fitting matrices are
+ * processed in chunks.  Results equal muon_ns_batched's.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current (cudaGetSymbolAddress) and caches it: make that first call
+ * before any stream capture.  Every call uses the same array, which keeps
+ * the previous call's contents (the call resets what must start at zero):
+ * calls that can overlap on the GPU (other streams, other host threads)
+ * race on it and must be serialised by the caller, e.g. on one stream. */
+#define MUON_NOALLOC_SCRATCH_BYTES (64u << 20)
+MUON_API int muon_ns_batched_noalloc(void* const* X, int count, int rows, int cols, int dtype,
+                                     const muon_ns_params* ns, int* status_per_matrix, void* stream);
+
 /* Algorithmic FLOPs of one orthogonalisation of a rows x cols matrix, every
  * product counted as 2 * rows * cols * inner [GramNS cost list]. */
 MUON_API double muon_ns_flops(int rows, int cols, const muon_ns_params* ns);

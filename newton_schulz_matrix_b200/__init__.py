@@ -21,7 +21,8 @@ __all__ = [
     "BF16", "FP16", "FP32", "STANDARD", "GRAM", "GRAM_STABILIZED", "QUINTIC", "CUBIC",
     "MuonError", "load_library", "library_path", "muon_step", "muon_ns_batched",
     "muon_workspace_size", "muon_workspace_min", "muon_ns_workspace_size", "muon_ns_flops",
-    "muon_status_string", "muon_profile_begin", "muon_profile_end", "MuonStep", "EXPORTED_SYMBOLS",
+    "muon_status_string", "muon_profile_begin", "muon_profile_end", "MuonStep", "muon_ns_batched_noalloc",
+    "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
 BF16, FP16, FP32 = 0, 1, 2
@@ -33,7 +34,9 @@ CUBIC = (1.5, -0.5, 0.0)
 EXPORTED_SYMBOLS = (
     "muon_workspace_size", "muon_workspace_min", "muon_step", "muon_ns_workspace_size",
     "muon_ns_batched", "muon_ns_flops", "muon_status_string", "muon_profile_begin", "muon_profile_end",
+    "muon_ns_batched_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB = None
@@ -94,6 +97,9 @@ def load_library() -> ctypes.CDLL:
     lib.muon_ns_batched.restype = ctypes.c_int
     lib.muon_ns_flops.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(_NSParams)]
     lib.muon_ns_flops.restype = ctypes.c_double
+    lib.muon_ns_batched_noalloc.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, ctypes.c_int, ctypes.POINTER(_NSParams), P, P]
+    lib.muon_ns_batched_noalloc.restype = ctypes.c_int
     lib.muon_profile_begin.argtypes = []
     lib.muon_profile_begin.restype = ctypes.c_int
     lib.muon_profile_end.argtypes = [ctypes.POINTER(_ProfEntry), ctypes.c_int]
@@ -336,3 +342,31 @@ class MuonStep:
         out = torch.empty_like(self.status)
         out[torch.tensor(self.order, device=out.device)] = self.status
         return out
+
+
+def muon_ns_batched_noalloc(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2,
+                            eps=1e-7, compute_dtype=None, gram_dtype="fp16", status: torch.Tensor | None = None,
+                            stream=None) -> None:
+    """muon_ns_batched with the library's fixed device scratch instead of a
+    workspace: for callers that cannot allocate device memory at this point
+    (their allocator owns the GPU, or allocation is forbidden after start-up).
+    Matrices whose one-matrix workspace exceeds NOALLOC_SCRATCH_BYTES are
+    rejected.  Calls share the scratch: do not let two of them overlap on the
+    GPU.  The first call on a device must come before any stream capture."""
+    lib = load_library()
+    if len(X) == 0:
+        return
+    for t in X:
+        _check_cuda(t, "X")
+        if t.shape != X[0].shape or t.dtype != X[0].dtype:
+            raise MuonError("all matrices must share shape and dtype")
+    rows, cols = X[0].shape
+    dt = _dtype_code(X[0].dtype)
+    if compute_dtype is None:
+        compute_dtype = "fp32" if dt == FP32 else "bf16"
+    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+    ptrs = (ctypes.c_void_p * len(X))(*[t.data_ptr() for t in X])
+    rc = lib.muon_ns_batched_noalloc(ptrs, len(X), rows, cols, dt, ctypes.byref(ns),
+                                     ctypes.c_void_p(status.data_ptr() if status is not None else 0),
+                                     ctypes.c_void_p(_stream_handle(stream)))
+    _raise(rc, "muon_ns_batched_noalloc")
