@@ -30,10 +30,9 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int round8(int v) { return (v + 7) / 8 * 8; }
 
 // ------------------------------------------------------------------ profiler
-enum ProfKind { kProfPack, kProfNorm, kProfConvert, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfKinds };
-const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "scale_convert_kernel",
-                                            "gemm_kernel[symmetric]", "gemm_kernel", "gemm_simt_kernel",
-                                            "unpack_kernel"};
+enum ProfKind { kProfPack, kProfNorm, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfKinds };
+const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "gemm_kernel[symmetric]", "gemm_kernel",
+                                            "gemm_simt_kernel", "unpack_kernel"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -197,32 +196,29 @@ GemmDesc desc(int M, int N, int K, int batch) {
   return g;
 }
 
-// Runs the Newton-Schulz chain on `chunk` packed matrices (raw U in X[0], in
-// bf16 for the tensor-core path, fp32 for the SIMT path).  Returns the index
-// of the X buffer that holds the result and the result's dtype.
+// Runs the Newton-Schulz chain on `chunk` packed matrices in X[0] and returns
+// the index of the X buffer that holds the result and the result's dtype.
 //
 // 16-bit chains: the standard form stores X, A, B in compute_dtype; the Gram
 // forms store every matrix of the chain (R, Q, Q_acc, X0, restart X) in
-// gram_dtype, so that no product mixes operand types.  A bf16 chain applies
-// the normalisation f = 1/(||U||+eps) inside the first products' epilogues;
-// an fp16 chain first writes X0 = f U in fp16 (fp16's range cannot hold an
-// arbitrary raw gradient).
-int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, int* out_x,
-              int* out_dtype) {
+// gram_dtype, so that no product mixes operand types.  A bf16 chain receives
+// the raw U (bf16's range holds any gradient) and applies f = 1/(||U||+eps)
+// inside the first products' epilogues; an fp16 chain receives X0 = f U
+// already normalised (`prescaled`), rounded once from fp32 to fp16.
+int chain_dtype(const muon_ns_params* ns) {
+  if (ns->compute_dtype == MUON_FP32) return MUON_FP32;
+  return ns->mode == MUON_NS_STANDARD ? ns->compute_dtype : ns->gram_dtype;
+}
+
+int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, bool prescaled,
+              int* out_x, int* out_dtype) {
   const int n = L.n, m = L.m, K = ns->iters;
-  const int cdt = c.compute == MUON_FP32 ? MUON_FP32
-                                         : (ns->mode == MUON_NS_STANDARD ? ns->compute_dtype : ns->gram_dtype);
+  const int cdt = chain_dtype(ns);
   const int xdt = cdt;  // X storage
   const int gdt = cdt;  // Gram-sized storage
   int rc;
-  int start = 0;
-  bool raw = true;
-  if (cdt == MUON_FP16) {
-    ProfScope ps(kProfConvert, 0.0, (double)chunk * B.x_bs * 4, c.s);
-    launch_scale_convert(B.X[0], B.X[1], B.inv, B.x_bs, chunk, c.s);
-    start = 1;
-    raw = false;
-  }
+  const int start = 0;
+  const bool raw = !prescaled;
   *out_dtype = xdt;
   if (ns->mode == MUON_NS_STANDARD) {
     int cur = start;
@@ -404,35 +400,48 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
         seg_i = si;
         seg_off = so;
       }
-      const int pack_dt = ns->compute_dtype == MUON_FP32 ? MUON_FP32 : MUON_BF16;
-      for (const Piece& pc : pieces) {
-        const SrcView& v = views[pc.group];
-        SegmentPtrs ptrs;
-        for (int i = 0; i < pc.count; ++i) {
-          ptrs.src[i] = v.src[pc.first + i];
-          ptrs.mom[i] = v.mom ? v.mom[pc.first + i] : nullptr;
-          ptrs.dst[i] = nullptr;
+      // fp16 chains take X0 normalised and rounded once to fp16: a sums-of-squares
+      // pass, the norm, then the storing pass with the scale.  Otherwise one pass
+      // stores the raw U (bf16 or fp32) and the chain applies the norm.
+      const int cdt = chain_dtype(ns);
+      const bool prescale = cdt == MUON_FP16;
+      const int pack_dt = ns->compute_dtype == MUON_FP32 ? MUON_FP32 : (prescale ? MUON_FP16 : MUON_BF16);
+      auto launch_pieces = [&](int pass) {
+        for (const Piece& pc : pieces) {
+          const SrcView& v = views[pc.group];
+          SegmentPtrs ptrs;
+          for (int i = 0; i < pc.count; ++i) {
+            ptrs.src[i] = v.src[pc.first + i];
+            ptrs.mom[i] = v.mom ? v.mom[pc.first + i] : nullptr;
+            ptrs.dst[i] = nullptr;
+          }
+          PackArgs a{};
+          a.rows = v.rows; a.cols = v.cols; a.count = pc.count;
+          a.src_dtype = v.src_dtype; a.x_dtype = pack_dt;
+          a.momentum_mode = update ? 1 : 0; a.mu = mu; a.nesterov = nesterov;
+          a.x = reinterpret_cast<char*>(B.X[0]) + (size_t)pc.slot * B.x_bs * L.x_es;
+          a.ld_x = L.ld_m; a.x_batch_stride = B.x_bs;
+          a.partials = B.partials + (size_t)pc.slot * L.tiles;
+          a.partial_stride = L.tiles;
+          a.pass = pass;
+          a.scale = B.inv + pc.slot;
+          const double elems = (double)v.rows * v.cols * pc.count;
+          const double in_b = dtype_size(v.src_dtype) + (update ? 4 : 0);
+          const double out_b = pass == 1 ? 0.0 : L.x_es + (update ? 4 : 0);
+          ProfScope ps(kProfPack, 0.0, elems * (in_b + out_b), s);
+          launch_pack(a, ptrs, s);
         }
-        PackArgs a{};
-        a.rows = v.rows; a.cols = v.cols; a.count = pc.count;
-        a.src_dtype = v.src_dtype; a.x_dtype = pack_dt;
-        a.momentum_mode = update ? 1 : 0; a.mu = mu; a.nesterov = nesterov;
-        a.x = reinterpret_cast<char*>(B.X[0]) + (size_t)pc.slot * B.x_bs * L.x_es;
-        a.ld_x = L.ld_m; a.x_batch_stride = B.x_bs;
-        a.partials = B.partials + (size_t)pc.slot * L.tiles;
-        a.partial_stride = L.tiles;
-        const double elems = (double)v.rows * v.cols * pc.count;
-        ProfScope ps(kProfPack, 0.0, elems * (dtype_size(v.src_dtype) + L.x_es + (update ? 8 : 0)), s);
-        launch_pack(a, ptrs, s);
-      }
+      };
+      launch_pieces(prescale ? 1 : 0);
       {
         ProfScope ps(kProfNorm, 0.0, (double)chunk * L.tiles * 4 + chunk * 4.0, s);
         launch_norm(B.partials, L.tiles, L.tiles, chunk, ns->eps, B.inv, s);
       }
+      if (prescale) launch_pieces(2);
       if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
       Ctx ctx{ns->compute_dtype, s, B.err};
       int xi = 0, out_dt = pack_dt;
-      if (run_chain(ctx, L, B, chunk, ns, &xi, &out_dt) != 0) return MUON_ERR_CUDA;
+      if (run_chain(ctx, L, B, chunk, ns, prescale, &xi, &out_dt) != 0) return MUON_ERR_CUDA;
       for (const Piece& pc : pieces) {
         const SrcView& v = views[pc.group];
         SegmentPtrs ptrs;

@@ -92,6 +92,7 @@ pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
   TX* x = reinterpret_cast<TX*>(a.x) + (long long)b * a.x_batch_stride;
 
   const bool full = (r0 + kTile <= a.rows) && (c0 + kTile <= a.cols) && (a.cols % 8 == 0);
+  const bool store = a.pass != 1;
   float u[16];
   float ssq = 0.f;
   if (full) {
@@ -106,7 +107,7 @@ pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
         m[i] = a.mu * m[i] + (1.f - a.mu) * g[i];
         u[i] = a.nesterov ? (1.f - a.mu) * g[i] + a.mu * m[i] : m[i];
       }
-      store16(mom + off, m);
+      if (store) store16(mom + off, m);
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i) u[i] = g[i];
@@ -121,7 +122,7 @@ pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
         float g = to_f32(src[off]);
         if (MOMENTUM) {
           float m = a.mu * mom[off] + (1.f - a.mu) * g;
-          mom[off] = m;
+          if (store) mom[off] = m;
           u[i] = a.nesterov ? (1.f - a.mu) * g + a.mu * m : m;
         } else {
           u[i] = g;
@@ -129,8 +130,20 @@ pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
       }
     }
   }
+  if (a.pass != 2) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) ssq += u[i] * u[i];
+    for (int i = 0; i < 16; ++i) ssq += u[i] * u[i];
+  }
+  if (a.pass == 1) {
+    const float s = block_sum_fixed(ssq, red);
+    if (threadIdx.x == 0) a.partials[(long long)b * a.partial_stride + blockIdx.x] = s;
+    return;
+  }
+  if (a.pass == 2) {
+    const float f = a.scale[b];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) u[i] *= f;
+  }
 
   if (!TRANS) {
     // oriented == storage: row r, columns c0 + lc ...
@@ -159,8 +172,10 @@ pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
         if (r0 + lc + i < a.rows) x[(long long)j * a.ld_x + r0 + lc + i] = from_f32<TX>(v[i]);
     }
   }
-  const float s = block_sum_fixed(ssq, red);
-  if (threadIdx.x == 0) a.partials[(long long)b * a.partial_stride + blockIdx.x] = s;
+  if (a.pass == 0) {
+    const float s = block_sum_fixed(ssq, red);
+    if (threadIdx.x == 0) a.partials[(long long)b * a.partial_stride + blockIdx.x] = s;
+  }
 }
 
 // ----------------------------------------------------------------------------
@@ -261,27 +276,6 @@ unpack_kernel(const UnpackArgs a, const __grid_constant__ SegmentPtrs p) {
 }
 
 // ----------------------------------------------------------------------------
-// normalise + convert: dst[b] = inv[b] * src[b] (bf16 -> fp16), 8 elements per
-// thread with 128-bit loads and stores; per_matrix is a multiple of 8
-// ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
-scale_convert_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, const float* __restrict__ inv,
-                     long long per_matrix, long long total) {
-  const long long n8 = total / 8;
-  for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8; v += (long long)gridDim.x * blockDim.x) {
-    const long long i = v * 8;
-    const float f = inv[i / per_matrix];
-    const uint4 q = reinterpret_cast<const uint4*>(src)[v];
-    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&q);
-    uint4 o;
-    __half* h = reinterpret_cast<__half*>(&o);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) h[k] = __float2half_rn(f * __bfloat162float(e[k]));
-    reinterpret_cast<uint4*>(dst)[v] = o;
-  }
-}
-
-// ----------------------------------------------------------------------------
 // dtype conversion of a flat array (rare Gram-mode corner cases)
 // ----------------------------------------------------------------------------
 __global__ void convert_kernel(const void* src, int sdt, void* dst, int ddt, long long n) {
@@ -357,17 +351,6 @@ void launch_unpack(const UnpackArgs& a, const SegmentPtrs& p, cudaStream_t s) {
     case kFP16: unpack_dispatch1<__half>(a, p, s); break;
     default: unpack_dispatch1<float>(a, p, s); break;
   }
-}
-
-void launch_scale_convert(const void* src, void* dst, const float* inv, long long per_matrix, int count,
-                          cudaStream_t s) {
-  const long long total = per_matrix * count;
-  if (total <= 0) return;
-  long long blocks = (total / 8 + 255) / 256;
-  const long long cap = (long long)num_sms() * 8;
-  if (blocks > cap) blocks = cap;
-  scale_convert_kernel<<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(src),
-                                                   reinterpret_cast<__half*>(dst), inv, per_matrix, total);
 }
 
 void launch_convert(const void* src, int sdt, void* dst, int ddt, long long n, cudaStream_t s) {

@@ -30,6 +30,11 @@ struct PackArgs {
   long long x_batch_stride;
   float* partials;      // [count][tiles] sums of squares, slot0 applied
   int partial_stride;   // partial entries per matrix
+  // pass 0: store M and raw U, write partials (one pass; the chain applies the norm)
+  // pass 1: write partials only (no stores): the first half of a normalised pack
+  // pass 2: store M and U * scale[b] (scale = 1/(||U||+eps) from pass 1), no partials
+  int pass;
+  const float* scale;   // pass 2: per-matrix factor, slot0 applied
 };
 int pack_tiles(int rows, int cols);
 void launch_pack(const PackArgs& a, const SegmentPtrs& p, cudaStream_t s);
@@ -52,10 +57,6 @@ struct UnpackArgs {
 };
 void launch_unpack(const UnpackArgs& a, const SegmentPtrs& p, cudaStream_t s);
 
-// dst[b] = inv[b] * src[b]: bf16 raw U -> fp16 X0 (per_matrix elements each,
-// a multiple of 8).
-void launch_scale_convert(const void* src, void* dst, const float* inv, long long per_matrix, int count,
-                          cudaStream_t s);
 void launch_convert(const void* src, int src_dtype, void* dst, int dst_dtype, long long n,
                     cudaStream_t s);
 
