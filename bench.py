@@ -36,6 +36,11 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "NS-orthogonalization ms/optimizer-step & effective TFLOP/s (% of bf16 peak)"
+# DRAM bytes (read + write) per product-kernel launch, averaged over the 45
+# launches of one Kimi-K2 step, from the ncu launch list summarised in
+# profiles/launches_kimi_k2_step.md.  Reset to None whenever the product
+# kernels change until a new capture is taken.
+PRODUCT_TRAFFIC_PER_LAUNCH = {"kimi-k2": 22.09e9}
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
@@ -152,8 +157,8 @@ class ClockSampler:
                 "power_w_max": max(num(r[3]) for r in rows)}
 
 
-def roofline_from_profile(prof, peaks, peak_kind):
-    gemm = [r for r in prof if r["kernel"].startswith("gemm_kernel")]
+def roofline_from_profile(prof, peaks, peak_kind, workload=None):
+    gemm = [r for r in prof if r["kernel"].startswith("tc_product")]
     if not gemm:
         return None
     fl = sum(r["flops"] for r in gemm)
@@ -161,11 +166,14 @@ def roofline_from_profile(prof, peaks, peak_kind):
     n = sum(r["launches"] for r in gemm)
     achieved = fl / (ms / 1e3) / 1e12
     peak = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
-    return {"bound": "tensor", "kernel": "gemm_kernel (tcgen05, all launches of the step)",
+    return {"bound": "tensor",
+            "kernel": "tcgen05 product kernels (gemm_pair_kernel, gemm_kernel below 256 rows), all launches of the step",
             "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
             "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
             "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
-            "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n, "traffic": None}
+            "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n,
+            "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get(workload),
+            "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per product launch (ncu, one step)"}
 
 
 def cpu_baseline_sample(w, hp, budget_s=20.0):
@@ -365,7 +373,7 @@ def main():
         cpu = cpu_baseline_sample(w, hp)
 
     if rank == 0:
-        roof = roofline_from_profile(prof, peaks, peak_kind)
+        roof = roofline_from_profile(prof, peaks, peak_kind, args.workload)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",

@@ -31,7 +31,8 @@ inline int round8(int v) { return (v + 7) / 8 * 8; }
 
 // ------------------------------------------------------------------ profiler
 enum ProfKind { kProfPack, kProfNorm, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfKinds };
-const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "gemm_kernel[symmetric]", "gemm_kernel",
+// product kinds cover both tensor-core kernels (gemm_pair_kernel for M >= 256, gemm_kernel below)
+const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "tc_product[symmetric]", "tc_product",
                                             "gemm_simt_kernel", "unpack_kernel"};
 struct ProfRec {
   int kind;
