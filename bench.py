@@ -58,6 +58,8 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-compare", action="store_true", help="skip the stabilised-Gram comparison run")
     p.add_argument("--workspace-gb", type=float, default=24.0, help="workspace cap (chunks the step beyond it)")
+    p.add_argument("--report", choices=["stress"], default=None,
+                   help="stress: the ill-conditioned sweep (one JSON line per (n, alpha) point) instead of the bench")
     return p.parse_args()
 
 
@@ -240,8 +242,76 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def sigma_band_device(U, O, coeffs, eps=1e-7):
+    """max |sigma_i(O) - f^K(sigma_i(U)/(||U||_F+eps))| via fp64 Gram eigenvalues on the device."""
+    import numpy as np
+    def svals(X):
+        X = X.double()
+        if X.shape[0] > X.shape[1]:
+            X = X.T
+        return torch.sqrt(torch.linalg.eigvalsh(X @ X.T).clamp_min(0)).cpu().numpy()
+    su, so = svals(U), svals(O)
+    t = su / (math.sqrt(float(np.sum(su * su))) + eps)
+    for a, b, c in coeffs:
+        t = a * t + b * t ** 3 + c * t ** 5
+    return float(np.max(np.abs(np.sort(so) - np.sort(t))))
+
+
+def run_stress_report(args):
+    """Ill-conditioned sweep: n in {1024, 2048, 4096}, alpha in {1, 2, 4, 8}, 32
+    matrices per point with log-uniform singular values in [1e-6, 1]; for each
+    form: device time, Inf/NaN count, sigma-band deviation (matrix 0, any size),
+    error against the fp64 oracle (matrix 0, n = 1024), FLOPs saved vs standard."""
+    import numpy as np
+    import newton_schulz_matrix_b200 as nsm
+    import synth
+    dev = torch.device("cuda", 0)
+    q5 = [synth.QUINTIC] * 5
+    for n in (1024, 2048, 4096):
+        for alpha in (1, 2, 4, 8):
+            mats = synth.stress_point(n, alpha, count=32, device=dev)
+            std_flops = nsm.muon_ns_flops(n, alpha * n)
+            line = {"report": "stress", "n": n, "alpha": alpha, "matrices": 32, "modes": {}}
+            for mode in ("standard", "gram", "gram_stabilized"):
+                ys = [m.clone() for m in mats]
+                ws = torch.empty(nsm.muon_ns_workspace_size(32, n, alpha * n, mode=mode), dtype=torch.uint8, device=dev)
+                st = torch.zeros(32, dtype=torch.int32, device=dev)
+                nsm.muon_ns_batched(ys, mode=mode, workspace=ws, status=st)
+                torch.cuda.synchronize()
+                bad = int((st != 0).sum())
+                finite0 = bool(torch.isfinite(ys[0]).all())
+                band = sigma_band_device(mats[0].float(), ys[0].float(), q5) if finite0 else None
+                err = None
+                if n == 1024 and finite0:
+                    import oracle
+                    U = mats[0].double().cpu().numpy()
+                    ref = oracle.newton_schulz(U, q5, mode=mode)
+                    err = float(np.linalg.norm(ys[0].double().cpu().numpy() - ref) / np.linalg.norm(ref))
+                ys2 = [m.clone() for m in mats]
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                nsm.muon_ns_batched(ys2, mode=mode, workspace=ws)
+                e0.record()
+                for _ in range(3):
+                    nsm.muon_ns_batched(ys2, mode=mode, workspace=ws)
+                e1.record()
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / 3
+                fl = nsm.muon_ns_flops(n, alpha * n, mode=mode)
+                line["modes"][mode] = {"ms": round(ms, 3), "nonfinite_matrices": bad, "sigma_band_dev": band,
+                                       "rel_err_vs_oracle": err, "flops": 32 * fl,
+                                       "flops_saved_vs_standard": round(1 - fl / std_flops, 4),
+                                       "effective_tflops": round(32 * fl / ms / 1e9, 1)}
+                del ys, ys2, ws
+            print(json.dumps(line), flush=True)
+            del mats
+            torch.cuda.empty_cache()
+
+
 def main():
     args = parse_args()
+    if args.report == "stress":
+        run_stress_report(args)
+        return
     if args.impl == "reference":
         run_reference(args)
         return
