@@ -63,6 +63,20 @@ def parse_args():
     return p.parse_args()
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The slowest rank's value (device-side all-reduce MAX); identity on one process."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Weak scaling: every rank runs the full workload; value = all ranks' FLOPs / max step time."""
+    return world * flops_per_rank_step / (ms_per_step / 1e3) / 1e12
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -365,13 +379,9 @@ def main():
     barrier()
     prof = nsm.muon_profile_end()
     clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    if dist is not None:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, device)
     status = step.status.cpu()
-    value = world * flops_step / (ms / 1e3) / 1e12
+    value = whole_job_tflops(world, flops_step, ms)
     launches_timed = sum(r["launches"] for r in prof)
 
     # stabilised Gram comparison on the same matrices (context for the Gram-vs-standard claim)
@@ -393,11 +403,7 @@ def main():
         c1.record(stream)
         torch.cuda.synchronize(device)
         barrier()
-        gms = c0.elapsed_time(c1) / nrep
-        if dist is not None:
-            t = torch.tensor([gms], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            gms = float(t.item())
+        gms = max_over_ranks(c0.elapsed_time(c1) / nrep, dist, device)
         compare = {"gram_stabilized_ms_per_step": round(gms, 3), "standard_ms_per_step": round(ms, 3),
                    "speedup_vs_standard": round(ms / gms, 3)}
         step = st2
@@ -405,7 +411,18 @@ def main():
     # end to end through the public API: gradients H2D from pinned host memory,
     # the step, updated weights D2H to pinned host memory, every step
     e2e = None
-    if not args.no_e2e:
+    # pinned host copies of G and W for every rank on this node must fit comfortably in RAM
+    local_world = int(os.environ.get("LOCAL_WORLD_SIZE", str(world)))
+    host_need = local_world * sum(t.numel() * t.element_size() for t in grads + params)
+    try:
+        import psutil
+        host_free = psutil.virtual_memory().available
+    except Exception:
+        host_free = 0
+    if not args.no_e2e and host_need > 0.6 * host_free:
+        e2e = {"value": None, "unit": "TFLOP/s", "skipped": f"pinned host buffers ({host_need / 2**30:.0f} GiB "
+               f"for {local_world} ranks) exceed 60% of free host memory ({host_free / 2**30:.0f} GiB)"}
+    elif not args.no_e2e:
         hG = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
         hW = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
         for h, g in zip(hG, grads):
@@ -428,12 +445,8 @@ def main():
         x1.record(stream)
         torch.cuda.synchronize(device)
         barrier()
-        ems = x0.elapsed_time(x1) / args.e2e_steps
-        if dist is not None:
-            t = torch.tensor([ems], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * flops_step / (ems / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": round(ems, 3),
+        ems = max_over_ranks(x0.elapsed_time(x1) / args.e2e_steps, dist, device)
+        e2e = {"value": whole_job_tflops(world, flops_step, ems), "unit": "TFLOP/s", "ms_per_step": round(ems, 3),
                "h2d_bytes_per_step": sum(g.numel() * g.element_size() for g in grads),
                "d2h_bytes_per_step": sum(p.numel() * p.element_size() for p in params)}
         del hG, hW

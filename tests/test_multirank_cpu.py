@@ -1,0 +1,105 @@
+"""Multi-process host logic on CPU with the gloo backend (world size 2):
+the bench's cross-rank timing reduction and weak-scaling value, and the
+sharded step's ownership plan and weight exchange (with an injected local
+update in place of the CUDA step)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from newton_schulz_matrix_b200.distributed import ShardedMuonStep, lpt_owners, ns_cost
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _init(rank, world, port):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+
+
+def _bench_worker(rank, world, port, q):
+    _init(rank, world, port)
+    import bench
+    ms = bench.max_over_ranks(100.0 + 10 * rank, dist, torch.device("cpu"))
+    v = bench.whole_job_tflops(world, 513.2e12, ms)
+    q.put((rank, ms, v))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def _sharded_worker(rank, world, port, q):
+    _init(rank, world, port)
+    torch.manual_seed(0)  # identical initial weights on every rank
+    shapes = [(64, 32), (16, 16), (128, 64), (32, 96), (8, 8), (64, 64), (48, 16)]
+    params = [torch.randn(*s) for s in shapes]
+    grads = [torch.randn(*s) for s in shapes]
+    start = [p.clone() for p in params]
+    owner = lpt_owners([ns_cost(s) for s in shapes], world)
+    moms = {i: torch.zeros(*shapes[i]) for i in range(len(shapes)) if owner[i] == rank}
+
+    def fake_local(ps, gs, ms, **hp):
+        def run():
+            for p, g in zip(ps, gs):
+                p.add_(g, alpha=1.0 + rank)   # rank-specific, so the broadcast source is visible
+        return run
+
+    step = ShardedMuonStep(params, grads, moms, local_step_factory=fake_local, lr=0.02)
+    assert step.owned() == [i for i, r in enumerate(owner) if r == rank]
+    step()
+    ok = all(torch.equal(params[i], start[i] + grads[i] * (1.0 + owner[i])) for i in range(len(shapes)))
+    q.put((rank, ok, owner))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def _spawn(fn, world=2):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=fn, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return sorted(out)
+
+
+def test_bench_timing_takes_the_slowest_rank():
+    out = _spawn(_bench_worker)
+    for rank, ms, v in out:
+        assert ms == 110.0
+        assert v == pytest.approx(2 * 513.2e12 / 0.110 / 1e12)
+
+
+def test_sharded_step_exchanges_owned_updates():
+    out = _spawn(_sharded_worker)
+    assert [ok for _, ok, _ in out] == [True, True]
+    assert out[0][2] == out[1][2]  # both ranks computed the same plan
+
+
+def test_lpt_balances_the_kimi_k2_set():
+    shapes = [(2048, 7168)] * 648 + [(7168, 18432)] * 3
+    costs = [ns_cost(s) for s in shapes]
+    for world in (2, 4, 8):
+        owner = lpt_owners(costs, world)
+        load = [0.0] * world
+        for c, r in zip(costs, owner):
+            load[r] += c
+        assert max(load) / (sum(load) / world) < 1.02
+        assert sorted(set(owner)) == list(range(world))
+    assert lpt_owners([5, 5, 5], 1) == [0, 0, 0]
+    with pytest.raises(ValueError):
+        lpt_owners([1.0], 0)
