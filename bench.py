@@ -58,6 +58,11 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-compare", action="store_true", help="skip the stabilised-Gram comparison run")
     p.add_argument("--workspace-gb", type=float, default=24.0, help="workspace cap (chunks the step beyond it)")
+    p.add_argument("--graph", action="store_true",
+                   help="replay the step from a CUDA graph (launch-latency-bound workloads such as 'single')")
+    p.add_argument("--sharded", action="store_true",
+                   help="strong scaling: shard one workload across the ranks (ownership by NS FLOPs, owner "
+                        "broadcast of the updated weights) instead of one full workload per rank")
     p.add_argument("--report", choices=["stress"], default=None,
                    help="stress: the ill-conditioned sweep (one JSON line per (n, alpha) point) instead of the bench")
     return p.parse_args()
@@ -112,7 +117,7 @@ def workload_config(w, params, mode, steps_note):
         shapes[k] = shapes.get(k, 0) + 1
     return {"workload": w.name, "matrices": len(params), "shapes": shapes, "mode": mode,
             "ns_iters": 5, "coeffs": [3.4445, -4.7750, 2.0315], "momentum": 0.95, "nesterov": True, "lr": 0.02,
-            "weight_decay": 0.1, "scale_coef": 0.2, "l2": steps_note, "parallelism": "replicas (weak)"}
+            "weight_decay": 0.1, "scale_coef": 0.2, "l2": steps_note}
 
 
 class ClockSampler:
@@ -333,7 +338,7 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     dist = None
-    if world > 1:
+    if world > 1 or (args.sharded and "MASTER_ADDR" in os.environ):
         import datetime
         import torch.distributed as dist
         torch.cuda.set_device(local)
@@ -347,12 +352,21 @@ def main():
     hp = dict(w.hp, mode=args.mode)
     compute = hp.get("compute_dtype", "bf16")
     ws_cap = int(args.workspace_gb * (1 << 30))
-    step = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, lr=hp["lr"], momentum=hp["momentum"],
-                        nesterov=hp["nesterov"], weight_decay=hp["weight_decay"], scale_coef=hp["scale_coef"],
-                        eps=hp["eps"], coeffs=hp["coeffs"], mode=hp["mode"], restart_after=hp["restart_after"],
-                        compute_dtype=compute)
+    step_hp = dict(lr=hp["lr"], momentum=hp["momentum"], nesterov=hp["nesterov"], weight_decay=hp["weight_decay"],
+                   scale_coef=hp["scale_coef"], eps=hp["eps"], coeffs=hp["coeffs"], mode=hp["mode"],
+                   restart_after=hp["restart_after"], compute_dtype=compute)
     flops_step = sum(nsm.muon_ns_flops(p.shape[0], p.shape[1], coeffs=hp["coeffs"], mode=hp["mode"],
                                        restart_after=hp["restart_after"]) for p in params)
+    if args.sharded:
+        if dist is None:
+            raise SystemExit("--sharded needs torchrun (one process per GPU)")
+        from newton_schulz_matrix_b200.distributed import ShardedMuonStep
+        owner_moms = {i: m for i, m in enumerate(moms)}
+        step = ShardedMuonStep(params, grads, owner_moms, local_step_factory=lambda ps, gs, ms, **h: nsm.MuonStep(
+            ps, gs, ms, workspace_bytes=ws_cap, **h), **step_hp)
+        flops_step /= world  # whole_job_tflops multiplies by world: the set is processed once in total
+    else:
+        step = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, **step_hp)
     resident = sum(t.numel() * t.element_size() for t in params + grads + moms)
     stream = torch.cuda.current_stream(device)
 
@@ -363,6 +377,15 @@ def main():
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
+    run = step
+    graph_launches = None
+    if args.graph and not args.sharded:
+        nsm.muon_profile_begin()
+        step()
+        torch.cuda.synchronize(device)
+        graph_launches = sum(r["launches"] for r in nsm.muon_profile_end())
+        graph = step.capture()
+        run = graph.replay
     clocks = ClockSampler(device)
     clocks.start()
     time.sleep(0.3)
@@ -373,20 +396,23 @@ def main():
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        run()
     e1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
     prof = nsm.muon_profile_end()
     clk = clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, device)
-    status = step.status.cpu()
+    status = step.local.status.cpu() if args.sharded and step.local is not None else (
+        torch.zeros(1, dtype=torch.int32) if args.sharded else step.status.cpu())
     value = whole_job_tflops(world, flops_step, ms)
-    launches_timed = sum(r["launches"] for r in prof)
+    launches_timed = sum(r["launches"] for r in prof) if graph_launches is None else graph_launches * args.steps
 
     # stabilised Gram comparison on the same matrices (context for the Gram-vs-standard claim)
     compare = None
-    if not args.no_compare and args.mode == "standard" and compute != "fp32":
+    if graph_launches is not None:
+        del run, graph
+    if not args.no_compare and args.mode == "standard" and compute != "fp32" and not args.sharded:
         del step
         torch.cuda.empty_cache()
         st2 = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, lr=hp["lr"], momentum=hp["momentum"],
@@ -422,16 +448,15 @@ def main():
     if not args.no_e2e and host_need > 0.6 * host_free:
         e2e = {"value": None, "unit": "TFLOP/s", "skipped": f"pinned host buffers ({host_need / 2**30:.0f} GiB "
                f"for {local_world} ranks) exceed 60% of free host memory ({host_free / 2**30:.0f} GiB)"}
-    elif not args.no_e2e:
+    elif not args.no_e2e and not args.sharded:
         hG = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
         hW = [torch.empty(p.shape, dtype=p.dtype, pin_memory=True) for p in params]
         for h, g in zip(hG, grads):
             h.copy_(g)
-        e2e_step = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, lr=hp["lr"], momentum=hp["momentum"],
-                                nesterov=hp["nesterov"], weight_decay=hp["weight_decay"], scale_coef=hp["scale_coef"],
-                                eps=hp["eps"], coeffs=hp["coeffs"], mode=hp["mode"],
-                                restart_after=hp["restart_after"], compute_dtype=compute)
         del step
+        torch.cuda.synchronize(device)
+        torch.cuda.empty_cache()
+        e2e_step = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, **step_hp)
         torch.cuda.synchronize(device)
         barrier()
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -459,10 +484,14 @@ def main():
         roof = roofline_from_profile(prof, peaks, peak_kind, args.workload)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "strong" if args.sharded else "weak",
             "vs_baseline": None, "dtype": "bf16" if compute != "fp32" else "f32",
             "data": "synthetic (seeded recipes of the workload; no datasets)",
-            "config": workload_config(w, params, hp["mode"], f"inputs larger than L2 ({resident / 2**30:.1f} GiB resident)"),
+            "config": dict(workload_config(w, params, hp["mode"], f"inputs larger than L2 ({resident / 2**30:.1f} GiB resident)"),
+                           parallelism=(f"sharded over {world} ranks (owner broadcast)" if args.sharded
+                                        else f"{world} replica(s), one full workload per GPU"),
+                           cuda_graph=bool(args.graph)),
             "pct_of_bf16_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
             "peaks": {"bf16_tflops": peaks["bf16_tflops"], "bf16_tflops_sustained": peaks.get("bf16_tflops_sustained"),
                       "source": peak_kind},

@@ -338,6 +338,22 @@ class MuonStep:
                                  ctypes.c_void_p(self.status.data_ptr()), ctypes.c_void_p(_stream_handle(stream)))
         _raise(rc, "muon_step")
 
+    def capture(self, stream=None) -> "torch.cuda.CUDAGraph":
+        """Record one step into a CUDA graph and return it; ``graph.replay()``
+        then runs the whole launch chain with one launch call.  The step is run
+        once eagerly first (one-time kernel set-up happens outside the capture),
+        so each capture advances the optimizer state by one step.  Inputs are
+        read from the same tensors at replay: update G in place between replays."""
+        side = torch.cuda.Stream(device=self.workspace.device) if stream is None else stream
+        side.wait_stream(torch.cuda.current_stream(self.workspace.device))
+        with torch.cuda.stream(side):
+            self(stream=side)
+        torch.cuda.current_stream(self.workspace.device).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            self(stream=side)
+        return g
+
     def status_in_param_order(self) -> torch.Tensor:
         out = torch.empty_like(self.status)
         out[torch.tensor(self.order, device=out.device)] = self.status

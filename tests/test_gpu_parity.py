@@ -269,3 +269,23 @@ def test_workspace_too_small_is_rejected():
     tiny = torch.empty(1024, dtype=torch.uint8, device=DEV)
     with pytest.raises(nsm.MuonError):
         nsm.muon_ns_batched([X], workspace=tiny)
+
+
+def test_captured_step_replays_the_eager_step():
+    """A step recorded in a CUDA graph and replayed gives the eager step's bits."""
+    spec = [(128, 384), (384, 128), (96, 200)]
+    for compute, wdt in (("bf16", torch.bfloat16), ("fp32", torch.float32)):
+        Wa, Ga, Ma = _groups_for_step(spec, wdt, 31)
+        Wb = [w.clone() for w in Wa]
+        Mb = [m.clone() for m in Ma]
+        eager = nsm.MuonStep(Wa, Ga, Ma, compute_dtype=compute)
+        graphed = nsm.MuonStep(Wb, Ga, Mb, compute_dtype=compute)
+        eager()                       # matches the capture's own eager warm-up step
+        g = graphed.capture()
+        for _ in range(3):
+            eager()
+            g.replay()
+        torch.cuda.synchronize()
+        for x, y in zip(Wa + Ma, Wb + Mb):
+            assert torch.equal(x, y)
+        assert int(graphed.status.abs().sum()) == 0
