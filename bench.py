@@ -53,6 +53,8 @@ def parse_args():
     p.add_argument("--workload", choices=["kimi-k2", "kimi-k2-experts16", "dense", "moe", "single"], default="kimi-k2",
                    help="kimi-k2-experts16: 16 expert matrices of the K2 set (small case for profiling)")
     p.add_argument("--mode", choices=["standard", "gram", "gram_stabilized"], default="standard")
+    p.add_argument("--compute", choices=["bf16", "fp16"], default=None,
+                   help="16-bit storage type of the standard chain (default: the workload's, bf16)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -351,6 +353,8 @@ def main():
     w, params, grads, moms = build_workload(args.workload, device)
     hp = dict(w.hp, mode=args.mode)
     compute = hp.get("compute_dtype", "bf16")
+    if args.compute is not None and compute != "fp32":
+        compute = args.compute
     ws_cap = int(args.workspace_gb * (1 << 30))
     step_hp = dict(lr=hp["lr"], momentum=hp["momentum"], nesterov=hp["nesterov"], weight_decay=hp["weight_decay"],
                    scale_coef=hp["scale_coef"], eps=hp["eps"], coeffs=hp["coeffs"], mode=hp["mode"],
@@ -486,7 +490,7 @@ def main():
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "strong" if args.sharded else "weak",
-            "vs_baseline": None, "dtype": "bf16" if compute != "fp32" else "f32",
+            "vs_baseline": None, "dtype": {"bf16": "bf16", "fp16": "f16", "fp32": "f32"}[compute],
             "data": "synthetic (seeded recipes of the workload; no datasets)",
             "config": dict(workload_config(w, params, hp["mode"], f"inputs larger than L2 ({resident / 2**30:.1f} GiB resident)"),
                            parallelism=(f"sharded over {world} ranks (owner broadcast)" if args.sharded

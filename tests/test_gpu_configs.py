@@ -207,3 +207,33 @@ def test_stress_sweep(n, alpha):
         assert rel(y0, want) < tolerance("bf16", floor), (mode, rel(y0, want), floor)
         if emulated_band_holds(U0, Q5, mode):
             assert sigma_band_error(U0, y0, Q5) < 0.05
+
+
+# ---------------------------------------------------------------------------
+# fp16 storage for the standard form meets the stated 2e-2 outright
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("workload", ["dense", "kimi-k2-subset"])
+def test_fp16_standard_meets_the_stated_tolerance(workload):
+    if workload == "dense":
+        w = synth.dense_projection(device=DEV, count=16)
+    else:
+        w = synth.kimi_k2(device=DEV, counts=[6, 3, 0, 0])
+    params, grads, moms, samples = [], [], [], []
+    for g in w.groups:
+        samples.append(len(params))
+        params += [x.float() for x in g.W]
+        grads += g.G
+        moms += g.M
+    W0 = {i: to_np(params[i]) for i in samples}
+    M0 = {i: to_np(moms[i]) for i in samples}
+    hp = step_hp()
+    status = run_step(params, grads, moms, mode="standard", compute_dtype="fp16", **hp)
+    assert int((status != 0).sum()) == 0
+    for i in samples:
+        r, c = params[i].shape
+        Wr, Mr, Or = oracle.muon_step(W0[i], to_np(grads[i]), M0[i], mode="standard", **hp)
+        step = hp["lr"] * hp["scale_coef"] * math.sqrt(max(r, c))
+        O = ((1 - hp["lr"] * hp["weight_decay"]) * W0[i] - to_np(params[i])) / step
+        assert rel(O, Or) < 2e-2
+        U = oracle.nesterov_blend(to_np(grads[i]), Mr, hp["momentum"], True)
+        assert sigma_band_error(U, O, Q5) < 0.05
