@@ -80,7 +80,7 @@ __device__ __forceinline__ float block_sum_fixed(float v, float* red) {
 template <typename TS, typename TX, bool MOMENTUM, bool TRANS>
 __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
-  __shared__ float tile[kTile][kTile + 1];
+  __shared__ float tile[TRANS ? kTile : 1][kTile + 1];
   __shared__ float red[kPackThreads / 32];
   const int b = blockIdx.y;
   const int tcols = (a.cols + kTile - 1) / kTile;
@@ -202,18 +202,23 @@ norm_kernel(const float* __restrict__ partials, int stride, int n, float eps, fl
 template <typename TD, typename TX, bool UPDATE, bool TRANS>
 __global__ void __launch_bounds__(kPackThreads)
 unpack_kernel(const UnpackArgs a, const __grid_constant__ SegmentPtrs p) {
-  __shared__ float tile[kTile][kTile + 1];
+  __shared__ float tile[TRANS ? kTile : 1][kTile + 1];
   const int b = blockIdx.y;
   const int tcols = (a.cols + kTile - 1) / kTile;
   const int r0 = (blockIdx.x / tcols) * kTile, c0 = (blockIdx.x % tcols) * kTile;
   const int lr = threadIdx.x >> 2, lc = (threadIdx.x & 3) * 16;
-  const TX* x = reinterpret_cast<const TX*>(a.x) + (long long)b * a.x_batch_stride;
-  TD* dst = reinterpret_cast<TD*>(p.dst[b]);
+  const TX* __restrict__ x = reinterpret_cast<const TX*>(a.x) + (long long)b * a.x_batch_stride;
+  TD* __restrict__ dst = reinterpret_cast<TD*>(p.dst[b]);
   const bool full = (r0 + kTile <= a.rows) && (c0 + kTile <= a.cols) && (a.cols % 8 == 0);
+  const int r = r0 + lr;
+  const long long off = (long long)r * a.cols + c0 + lc;
 
+  // Both global loads (W and the orientated O) are issued before either is used,
+  // so each thread waits for one memory round trip, not two.
+  float w[16];
+  if (UPDATE && full) load16(dst + off, w);
   float o[16];
   if (!TRANS) {
-    const int r = r0 + lr;
     if (full) {
       load16(x + (long long)r * a.ld_x + c0 + lc, o);
     } else {
@@ -239,16 +244,8 @@ unpack_kernel(const UnpackArgs a, const __grid_constant__ SegmentPtrs p) {
     for (int i = 0; i < 16; ++i) o[i] = tile[lc + i][lr];
   }
 
-  int bad = 0;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) bad |= !isfinite(o[i]);
-
-  const int r = r0 + lr;
   if (full) {
-    const long long off = (long long)r * a.cols + c0 + lc;
-    float w[16];
     if (UPDATE) {
-      load16(dst + off, w);
 #pragma unroll
       for (int i = 0; i < 16; ++i) w[i] = a.decay * w[i] - a.step * o[i];
     } else {
@@ -261,17 +258,23 @@ unpack_kernel(const UnpackArgs a, const __grid_constant__ SegmentPtrs p) {
     for (int i = 0; i < 16; ++i) {
       const int c = c0 + lc + i;
       if (c < a.cols) {
-        const long long off = (long long)r * a.cols + c;
-        float w = UPDATE ? a.decay * to_f32(dst[off]) - a.step * o[i] : o[i];
-        dst[off] = from_f32<TD>(w);
+        const long long o2 = (long long)r * a.cols + c;
+        float v = UPDATE ? a.decay * to_f32(dst[o2]) - a.step * o[i] : o[i];
+        dst[o2] = from_f32<TD>(v);
       }
     }
   }
-  bad = __syncthreads_or(bad);
-  if (threadIdx.x == 0 && a.status != nullptr) {
-    int st = bad ? kStatusNonFinite : 0;
-    if (blockIdx.x == 0 && a.chunk_err != nullptr) st |= *a.chunk_err;
-    if (st) atomicOr(a.status + b, st);
+
+  if (a.status != nullptr) {
+    int bad = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) bad |= !isfinite(o[i]);
+    bad = __any_sync(0xffffffffu, bad);
+    if ((threadIdx.x & 31) == 0) {
+      int st = bad ? kStatusNonFinite : 0;
+      if (blockIdx.x == 0 && threadIdx.x == 0 && a.chunk_err != nullptr) st |= *a.chunk_err;
+      if (st) atomicOr(a.status + b, st);
+    }
   }
 }
 

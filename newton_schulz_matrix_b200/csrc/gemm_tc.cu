@@ -33,13 +33,14 @@ namespace muon {
 namespace tc {
 
 // ------------------------------------------------------------------ kernel
-template <bool B_MN, int IN_FMT>
+template <bool B_MN, int IN_FMT, bool SYM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+            const __grid_constant__ CUtensorMap tmap_d,
             const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint16_t* staging = reinterpret_cast<uint16_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* staging = smem + STAGES * STAGE_BYTES;  // per epilogue warp: two 1024-aligned 2 KB boxes
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + STAGING_BYTES);
   uint64_t* full_bar = bars;                    // [STAGES]
   uint64_t* empty_bar = bars + STAGES;          // [STAGES]
@@ -68,6 +69,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_d)) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -158,7 +160,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
     // ---------------------------------------------------------------- epilogue
     const int q = warp & 3;                      // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;            // which 4 of the 8 column chunks
-    uint16_t* stage = staging + (warp - 2) * (STAGE_BYTES_PER_WARP / 2);
+    uint8_t* S = staging + (warp - 2) * 2 * STAGE_TILE_BYTES;
+    uint8_t* T = S + STAGE_TILE_BYTES;
     int it = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++it) {
       const Tile tl = decode_tile(p, t);
@@ -192,9 +195,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ 
           tc_fence_before();
           mbar_arrive(smem_u32(&tempty_bar[acc]));
         }
-        epilogue_chunk(p, tl, q, lane, c, r, creg, c_ready, f, stage);
+        epilogue_chunk<SYM>(p, &tmap_d, tl, q, lane, c, r, creg, c_ready, f, S, T);
       }
     }
+    if (lane == 0) bulk_wait_all0();  // this warp's output stores have completed
+    __syncwarp();
   }
 
   __syncwarp();
@@ -226,8 +231,8 @@ static EncodeTiledFn get_encode() {
 }
 
 // 3-D tiled map over a batch of row-major matrices: dims (inner, outer, batch).
-bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer,
-                       long long batch, long long ld_elems, long long bs_elems, int box_inner, int box_outer) {
+bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer, long long batch,
+                long long ld_elems, long long bs_elems, int box_inner, int box_outer, int swizzle_bytes) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   const CUtensorMapDataType dt = dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -235,22 +240,28 @@ bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, 
   cuuint64_t strides[2] = {(cuuint64_t)ld_elems * 2, (cuuint64_t)(bs_elems > 0 ? bs_elems : ld_elems * outer) * 2};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer, 1};
   cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <bool B_MN, int IN_FMT>
-static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+bool encode_out_map(CUtensorMap* map, const GemmDesc& g) {
+  return encode_map(map, g.d_dtype, g.D, g.N, g.M, g.batch, g.ldd, g.d_bs, 32, 32, 64);
+}
+
+template <bool B_MN, int IN_FMT, bool SYM>
+static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
+                  cudaStream_t s) {
   static bool attr_done = false;
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<B_MN, IN_FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<B_MN, IN_FMT, SYM>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return (int)e;
     attr_done = true;
   }
   const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
-  gemm_kernel<B_MN, IN_FMT><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+  gemm_kernel<B_MN, IN_FMT, SYM><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, md, p);
   return (int)cudaGetLastError();
 }
 
@@ -301,9 +312,15 @@ int gemm_tc(const GemmDesc& g, cudaStream_t s) {
   } else {
     if (!encode_map(&mb, g.in_dtype, g.B, g.K, g.N, g.batch, g.ldb, g.b_bs, BK, BN)) return (int)cudaErrorInvalidValue;
   }
+  CUtensorMap md;
+  if (!encode_out_map(&md, g)) return (int)cudaErrorInvalidValue;
   const int fmt = g.in_dtype == kBF16 ? 1 : 0;
-  if (bmn) return fmt ? launch<true, 1>(ma, mb, p, s) : launch<true, 0>(ma, mb, p, s);
-  return fmt ? launch<false, 1>(ma, mb, p, s) : launch<false, 0>(ma, mb, p, s);
+  if (g.symmetric) {
+    if (bmn) return fmt ? launch<true, 1, true>(ma, mb, md, p, s) : launch<true, 0, true>(ma, mb, md, p, s);
+    return fmt ? launch<false, 1, true>(ma, mb, md, p, s) : launch<false, 0, true>(ma, mb, md, p, s);
+  }
+  if (bmn) return fmt ? launch<true, 1, false>(ma, mb, md, p, s) : launch<true, 0, false>(ma, mb, md, p, s);
+  return fmt ? launch<false, 1, false>(ma, mb, md, p, s) : launch<false, 0, false>(ma, mb, md, p, s);
 }
 
 int num_sms() {

@@ -97,13 +97,14 @@ __device__ __forceinline__ PairTile decode_pair(const Params& p, int t) {
   return r;
 }
 
-template <bool B_MN, int IN_FMT>
+template <bool B_MN, int IN_FMT, bool SYM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+            const __grid_constant__ CUtensorMap tmap_d,
                  const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint16_t* staging = reinterpret_cast<uint16_t*>(smem + STAGES2 * STAGE_BYTES2);
+  uint8_t* staging = smem + STAGES2 * STAGE_BYTES2;  // per epilogue warp: two 1024-aligned 2 KB boxes
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES2 * STAGE_BYTES2 + STAGING_BYTES);
   uint64_t* full_bar = bars;                      // [STAGES2]   (used in the leader)
   uint64_t* empty_bar = bars + STAGES2;           // [STAGES2]   (both CTAs)
@@ -135,6 +136,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_d)) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -220,7 +222,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     // ---------------------------------------------------------------- epilogue (both CTAs)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
-    uint16_t* stage = staging + (warp - 2) * (STAGE_BYTES_PER_WARP / 2);
+    uint8_t* S = staging + (warp - 2) * 2 * STAGE_TILE_BYTES;
+    uint8_t* T = S + STAGE_TILE_BYTES;
     int it = 0;
     for (int t = pair; t < p.total_tiles; t += npairs, ++it) {
       const PairTile pt = decode_pair(p, t);
@@ -255,9 +258,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           __syncwarp();
           if (lane == 0) remote_arrive(leader_tempty + acc * 8);
         }
-        epilogue_chunk(p, tl, q, lane, c, r, creg, c_ready, f, stage);
+        epilogue_chunk<SYM>(p, &tmap_d, tl, q, lane, c, r, creg, c_ready, f, S, T);
       }
     }
+    if (lane == 0) bulk_wait_all0();  // this warp's output stores have completed
+    __syncwarp();
   }
 
   __syncwarp();
@@ -271,10 +276,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   if (threadIdx.x == 0 && *abort_flag && p.err != nullptr) atomicOr(p.err, kStatusTimeout);
 }
 
-template <bool B_MN, int IN_FMT>
-static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+template <bool B_MN, int IN_FMT, bool SYM>
+static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
+                  cudaStream_t s) {
   static int max_pairs = 0;
-  auto kern = gemm_pair_kernel<B_MN, IN_FMT>;
+  auto kern = gemm_pair_kernel<B_MN, IN_FMT, SYM>;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -297,7 +303,7 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p,
   }
   const int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   cfg.gridDim = dim3(2 * pairs);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p);
   return (int)e;
 }
 
@@ -324,9 +330,15 @@ int gemm_tc_pair(const GemmDesc& g, Params p, cudaStream_t s) {
   } else {
     if (!encode_map(&mb, g.in_dtype, g.B, g.K, g.N, g.batch, g.ldb, g.b_bs, BK, 128)) return (int)cudaErrorInvalidValue;
   }
+  CUtensorMap md;
+  if (!encode_out_map(&md, g)) return (int)cudaErrorInvalidValue;
   const int fmt = g.in_dtype == kBF16 ? 1 : 0;
-  if (bmn) return fmt ? launch<true, 1>(ma, mb, p, s) : launch<true, 0>(ma, mb, p, s);
-  return fmt ? launch<false, 1>(ma, mb, p, s) : launch<false, 0>(ma, mb, p, s);
+  if (g.symmetric) {
+    if (bmn) return fmt ? launch<true, 1, true>(ma, mb, md, p, s) : launch<true, 0, true>(ma, mb, md, p, s);
+    return fmt ? launch<false, 1, true>(ma, mb, md, p, s) : launch<false, 0, true>(ma, mb, md, p, s);
+  }
+  if (bmn) return fmt ? launch<true, 1, false>(ma, mb, md, p, s) : launch<true, 0, false>(ma, mb, md, p, s);
+  return fmt ? launch<false, 1, false>(ma, mb, md, p, s) : launch<false, 0, false>(ma, mb, md, p, s);
 }
 
 }  // namespace tc

@@ -23,7 +23,8 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_EPI_WARPS = 8;         // two per TMEM lane quarter, 4 chunks of 32 columns each
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int TMEM_COLS = 2 * BN;        // two fp32 accumulators
-constexpr int STAGING_BYTES = NUM_EPI_WARPS * 32 * 40 * 2;  // mirrored-store staging tiles
+constexpr int STAGE_TILE_BYTES = 32 * 32 * 2;                     // one 32 x 32 16-bit output box
+constexpr int STAGING_BYTES = NUM_EPI_WARPS * 2 * STAGE_TILE_BYTES;  // per epilogue warp: direct + transposed box
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STAGING_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int GROUP_M = 8;               // tile raster grouping for L2 reuse
 
@@ -176,25 +177,6 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
 }
 
 // ------------------------------------------------------------------ epilogue
-__device__ __forceinline__ void store_row32(void* D, int dt, long long off, const float* v) {
-  uint4 q[4];
-  if (dt == kBF16) {
-    __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(q);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) e[i] = __float2bfloat16_rn(v[i]);
-    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(D) + off);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = q[i];
-  } else {
-    __half* e = reinterpret_cast<__half*>(q);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) e[i] = __float2half_rn(v[i]);
-    uint4* d = reinterpret_cast<uint4*>(reinterpret_cast<__half*>(D) + off);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) d[i] = q[i];
-  }
-}
-
 __device__ __forceinline__ void cvt_row32(const uint4 (&q)[4], int dt, float* v) {
   if (dt == kBF16) {
     const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -212,30 +194,67 @@ __device__ __forceinline__ uint16_t to_bits(float v, int dt) {
   return __half_as_ushort(__float2half_rn(v));
 }
 
-// Per-warp shared staging tile for the mirrored (transposed) store of one
-// 32 x 32 chunk: 32 rows of 40 halfwords (80-byte stride keeps the row-wise
-// 16-byte reads free of bank conflicts).
-constexpr int STAGE_LD = 40;
-constexpr int STAGE_BYTES_PER_WARP = 32 * STAGE_LD * 2;
+// ------------------------------------------------------------------ epilogue stores via TMA
+// A warp writes one 32 x 32 output box into shared memory in the layout of a
+// 64-byte-swizzled tensor map (row r, 16-byte chunk k at r*64 + ((k ^ (r>>1 & 3)) << 4),
+// conflict-free for both row-wise and column-wise writes), and one lane hands it to
+// the TMA unit with a bulk tensor store, which also clips rows and columns past
+// the matrix edge.
+__device__ __forceinline__ uint32_t sw64(int row, int chunk16) {
+  return (uint32_t)(row * 64 + ((chunk16 ^ ((row >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void pack_row32(const float* v, int dt, uint4 (&q)[4]) {
+  if (dt == kBF16) {
+    __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) e[i] = __float2bfloat16_rn(v[i]);
+  } else {
+    __half* e = reinterpret_cast<__half*>(q);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) e[i] = __float2half_rn(v[i]);
+  }
+}
 
 // One 32 x 32 chunk of the output: this warp's 32 tile rows (one per lane,
 // TMEM lane quarter q) times columns [gj0, gj0 + 32).  `creg` holds the C row
 // segment when `c_ready` (loaded before the TMEM read to hide its latency).
-__device__ __forceinline__ void epilogue_chunk(const Params& p, const Tile& t, int q, int lane, int chunk,
-                                               const uint32_t (&acc)[32], const uint4 (&creg)[4], bool c_ready,
-                                               float f, uint16_t* stage) {
+// Symmetric products: off-diagonal 128-blocks are stored directly and
+// transposed; inside a diagonal 128-block, boxes above the diagonal are stored
+// both ways, boxes below are skipped (their transposes cover them) and the box
+// on the diagonal is made exactly symmetric in shared memory first.
+// S and T are this warp's two staging boxes (1024-byte aligned).
+template <bool SYM>
+__device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMap* tmap_d, const Tile& t, int q,
+                                               int lane, int chunk, const uint32_t (&acc)[32],
+                                               const uint4 (&creg)[4], bool c_ready, float f, uint8_t* S,
+                                               uint8_t* T) {
   const int gi_base = t.tm * BM + q * 32;
   const int gi = gi_base + lane;
   const int gj0 = t.tn * BN + chunk * 32;
-  // 0: plain store; 1: store + mirror; 2: diagonal block (upper half + mirror)
-  int kind = 0;
-  if (p.symmetric) {
+  bool mirror = false, diag_box = false;
+  if (SYM) {
     const int bj = t.tn * 2 + (chunk >> 2);  // 128-column block of this chunk
-    if (bj < t.tm) return;                   // lower block: stored as the mirror of its transpose
-    kind = bj > t.tm ? 1 : 2;
+    if (bj < t.tm) return;                   // lower block: stored as the transpose of its mirror
+    if (bj > t.tm) {
+      mirror = true;
+    } else {                                 // diagonal 128-block
+      if (gj0 < gi_base) return;             // box below the diagonal
+      diag_box = gj0 == gi_base;
+      mirror = !diag_box;
+    }
   }
   if (gj0 >= p.N || gi_base >= p.M) return;  // warp-uniform
-  const bool full = gj0 + 32 <= p.N;
   float v[32];
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = p.c_acc * __uint_as_float(acc[j]);
@@ -259,51 +278,52 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const Tile& t, i
     if (gj0 + j == gi) v[j] += p.c_eye;
   }
 
-  char* db = reinterpret_cast<char*>(p.D) + (long long)t.b * p.d_bs * 2;
-  // direct store of row gi (diagonal blocks: only columns >= gi)
-  if (gi < p.M) {
-    const long long off = (long long)gi * p.ldd + gj0;
-    if (full && (kind != 2 || gj0 >= gi)) {
-      store_row32(db, p.d_dtype, off, v);
-    } else {
+  // the staging boxes are free once the previous chunk's stores have read them
+  if (lane == 0) bulk_wait_read0();
+  __syncwarp();
+  if (SYM && (mirror || diag_box)) {
+    // transposed box: T[j][lane] = v[j]
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      *reinterpret_cast<uint16_t*>(T + sw64(j, lane >> 3) + (lane & 7) * 2) = to_bits(v[j], p.d_dtype);
+    if (diag_box) {
+      __syncwarp();
+      // below the diagonal take the transposed value, so the box is exactly symmetric
+      uint4 tq[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) tq[k] = *reinterpret_cast<const uint4*>(T + sw64(lane, k));
+      const uint16_t* te = reinterpret_cast<const uint16_t*>(tq);
+      uint4 dq[4];
+      pack_row32(v, p.d_dtype, dq);
+      uint16_t* de = reinterpret_cast<uint16_t*>(dq);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        if (gj0 + j < p.N && (kind != 2 || gj0 + j >= gi)) store_any(db, off + j, p.d_dtype, v[j]);
+        if (j < lane) de[j] = te[j];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(S + sw64(lane, k)) = dq[k];
     }
   }
-  if (kind == 0) return;
-  // mirrored store D[gj][gi] through the staging tile: lane l writes target row gj0 + l
+  if (!diag_box) {
+    uint4 dq[4];
+    pack_row32(v, p.d_dtype, dq);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(S + sw64(lane, k)) = dq[k];
+  }
+  fence_async_smem();
   __syncwarp();
-#pragma unroll
-  for (int j = 0; j < 32; ++j) stage[j * STAGE_LD + lane] = to_bits(v[j], p.d_dtype);
-  __syncwarp();
-  const int row = gj0 + lane;
-  if (row < p.N) {
-    uint4 w[4];
-    const uint4* src = reinterpret_cast<const uint4*>(stage + lane * STAGE_LD);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) w[i] = src[i];
-    uint16_t* drow = reinterpret_cast<uint16_t*>(db) + (long long)row * p.ldd + gi_base;
-    // valid columns: gi_base + k < M, and for diagonal blocks strictly below the diagonal (k < row - gi_base)
-    const int lim_m = p.M - gi_base;
-    const int lim = kind == 2 ? min(lim_m, row - gi_base) : lim_m;
-    if (lim >= 32) {
-      uint4* d = reinterpret_cast<uint4*>(drow);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) d[i] = w[i];
-    } else {
-      const uint16_t* e = reinterpret_cast<const uint16_t*>(w);
-#pragma unroll
-      for (int k = 0; k < 32; ++k)
-        if (k < lim) drow[k] = e[k];
-    }
+  if (lane == 0) {
+    tma_store_3d(tmap_d, smem_u32(S), gj0, gi_base, t.b);
+    if (SYM && mirror) tma_store_3d(tmap_d, smem_u32(T), gi_base, gj0, t.b);
+    bulk_commit();
   }
 }
 
 // ------------------------------------------------------------------ host side (gemm_tc.cu)
 // 3-D tiled tensor map over a batch of row-major matrices, 128-byte swizzle.
 bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer, long long batch,
-                long long ld_elems, long long bs_elems, int box_inner, int box_outer);
+                long long ld_elems, long long bs_elems, int box_inner, int box_outer, int swizzle_bytes = 128);
+// Output map of a product: 32 x 32 boxes, 64-byte swizzle (the epilogue's staging layout).
+bool encode_out_map(CUtensorMap* map, const GemmDesc& g);
 // 2-CTA (cta_group::2) variant for 256-row tiles (gemm_tc2.cu).
 int gemm_tc_pair(const GemmDesc& g, Params p, cudaStream_t s);
 
