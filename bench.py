@@ -40,7 +40,7 @@ METRIC = "NS-orthogonalization ms/optimizer-step & effective TFLOP/s (% of bf16 
 # launches of one Kimi-K2 step, from the ncu launch list summarised in
 # profiles/launches_kimi_k2_step.md.  Reset to None whenever the product
 # kernels change until a new capture is taken.
-PRODUCT_TRAFFIC_PER_LAUNCH = {"kimi-k2": None}
+PRODUCT_TRAFFIC_PER_LAUNCH = {"kimi-k2": 20.79e9}
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 

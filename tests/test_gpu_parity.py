@@ -289,3 +289,25 @@ def test_captured_step_replays_the_eager_step():
         for x, y in zip(Wa + Ma, Wb + Mb):
             assert torch.equal(x, y)
         assert int(graphed.status.abs().sum()) == 0
+
+
+def test_checkpoint_resume_is_bit_identical():
+    """The only optimizer state is M (owned by the caller): saving W and M,
+    stepping, restoring and stepping again reproduces the same bits."""
+    spec = [(256, 768), (768, 256), (130, 520)]
+    for mode in ("standard", "gram_stabilized"):
+        Ws, Gs, Ms = _groups_for_step(spec, torch.bfloat16, 41)
+        nsm.muon_step(Ws, Gs, Ms, mode=mode)
+        saved_W = [w.clone() for w in Ws]
+        saved_M = [m.clone() for m in Ms]
+        nsm.muon_step(Ws, Gs, Ms, mode=mode)
+        after_W = [w.clone() for w in Ws]
+        after_M = [m.clone() for m in Ms]
+        for w, s in zip(Ws, saved_W):
+            w.copy_(s)
+        for m, s in zip(Ms, saved_M):
+            m.copy_(s)
+        nsm.muon_step(Ws, Gs, Ms, mode=mode)
+        torch.cuda.synchronize()
+        for x, y in zip(Ws + Ms, after_W + after_M):
+            assert torch.equal(x, y)
