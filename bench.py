@@ -460,17 +460,16 @@ def main():
         del step
         torch.cuda.synchronize(device)
         torch.cuda.empty_cache()
-        e2e_step = nsm.MuonStep(params, grads, moms, workspace_bytes=ws_cap, **step_hp)
+        # gradients stream in from pinned host memory and updated weights stream out,
+        # slice by slice, overlapped with the orthogonalisation of other slices
+        e2e_step = nsm.StreamedMuonStep(params, grads, moms, hG, hW, workspace_bytes=ws_cap, **step_hp)
+        e2e_step()
         torch.cuda.synchronize(device)
         barrier()
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         x0.record(stream)
         for _ in range(args.e2e_steps):
-            for d, h in zip(grads, hG):
-                d.copy_(h, non_blocking=True)
             e2e_step()
-            for h, d in zip(hW, params):
-                h.copy_(d, non_blocking=True)
         x1.record(stream)
         torch.cuda.synchronize(device)
         barrier()

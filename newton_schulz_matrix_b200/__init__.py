@@ -21,7 +21,8 @@ __all__ = [
     "BF16", "FP16", "FP32", "STANDARD", "GRAM", "GRAM_STABILIZED", "QUINTIC", "CUBIC",
     "MuonError", "load_library", "library_path", "muon_step", "muon_ns_batched",
     "muon_workspace_size", "muon_workspace_min", "muon_ns_workspace_size", "muon_ns_flops",
-    "muon_status_string", "muon_profile_begin", "muon_profile_end", "MuonStep", "muon_ns_batched_noalloc",
+    "muon_status_string", "muon_profile_begin", "muon_profile_end", "MuonStep", "StreamedMuonStep",
+    "muon_ns_batched_noalloc",
     "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
@@ -318,7 +319,8 @@ class MuonStep:
     must stay alive and keep their storage for the object's lifetime.
     """
 
-    def __init__(self, params, grads, moms, *, workspace_bytes: int | None = None, **hp):
+    def __init__(self, params, grads, moms, *, workspace_bytes: int | None = None,
+                 workspace: torch.Tensor | None = None, **hp):
         self._lib = load_library()
         a = dict(_STEP_DEFAULTS, **hp)
         self.hp = a
@@ -327,8 +329,14 @@ class MuonStep:
         lo = int(self._lib.muon_workspace_min(self._groups, self._ng, ctypes.byref(self._h)))
         if full == 0:
             raise MuonError("invalid arguments (workspace query returned 0)")
-        size = full if workspace_bytes is None else max(lo, min(full, int(workspace_bytes)))
-        self.workspace = torch.empty(size, dtype=torch.uint8, device=params[0].device)
+        self.workspace_needed = (lo, full)
+        if workspace is not None:
+            if workspace.numel() * workspace.element_size() < lo:
+                raise MuonError(f"workspace of {workspace.numel()} bytes is below the minimum {lo}")
+            self.workspace = workspace
+        else:
+            size = full if workspace_bytes is None else max(lo, min(full, int(workspace_bytes)))
+            self.workspace = torch.empty(size, dtype=torch.uint8, device=params[0].device)
         self.status = torch.zeros(len(self.order), dtype=torch.int32, device=params[0].device)
         self.count = len(self.order)
 
@@ -386,3 +394,89 @@ def muon_ns_batched_noalloc(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5,
                                      ctypes.c_void_p(status.data_ptr() if status is not None else 0),
                                      ctypes.c_void_p(_stream_handle(stream)))
     _raise(rc, "muon_ns_batched_noalloc")
+
+
+class StreamedMuonStep:
+    """A Muon step fed from and returned to pinned host memory, with the PCIe
+    copies overlapped with the orthogonalisation.
+
+    The parameters are cut into slices of consecutive tensors (at most
+    ``slice_bytes`` of gradients each).  Per slice, one stream copies the
+    gradients host -> device, the compute stream runs the fused step on the
+    slice, and a third stream copies the updated weights device -> host, so
+    slice k's step runs while slice k+1's gradients arrive and slice k-1's
+    weights leave.  Every slice shares one workspace (the steps are serialised
+    on the compute stream).  Across calls, a slice's gradient buffer is not
+    overwritten before the previous step has read it, nor its weights updated
+    before the previous copy-out has read them.  The caller's current stream
+    waits for the whole step at the end of each call.
+    """
+
+    def __init__(self, params, grads, moms, host_grads, host_params, *, slice_bytes: int = 2 << 30,
+                 workspace_bytes: int | None = None, **hp):
+        if not (len(params) == len(grads) == len(moms) == len(host_grads) == len(host_params)):
+            raise MuonError("params, grads, moms and their host copies must have equal lengths")
+        for h in list(host_grads) + list(host_params):
+            if h.is_cuda or not h.is_pinned():
+                raise MuonError("host buffers must be pinned CPU tensors")
+        dev = params[0].device
+        self.params, self.grads = list(params), list(grads)
+        self.host_grads, self.host_params = list(host_grads), list(host_params)
+        self.slices = []
+        start, acc = 0, 0
+        for i, g in enumerate(self.grads):
+            b = g.numel() * g.element_size()
+            if i > start and acc + b > slice_bytes:
+                self.slices.append((start, i))
+                start, acc = i, 0
+            acc += b
+        self.slices.append((start, len(self.grads)))
+        self.steps = [MuonStep(self.params[a:b], self.grads[a:b], list(moms[a:b]), workspace=None,
+                               workspace_bytes=1, **hp) for a, b in self.slices]
+        need = max(st.workspace_needed[1] for st in self.steps)
+        if workspace_bytes is not None:
+            need = max(max(st.workspace_needed[0] for st in self.steps), min(need, int(workspace_bytes)))
+        self.workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        for st in self.steps:
+            st.workspace = self.workspace
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.compute = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        n = len(self.slices)
+        self._computed = [None] * n   # event: slice's step finished (its gradients are read)
+        self._copied_out = [None] * n  # event: slice's weights are on the host
+
+    def __call__(self) -> None:
+        caller = torch.cuda.current_stream(self.workspace.device)
+        for s in (self.h2d, self.compute, self.d2h):
+            s.wait_stream(caller)
+        done = []
+        for k, (a, b) in enumerate(self.slices):
+            with torch.cuda.stream(self.h2d):
+                if self._computed[k] is not None:
+                    self.h2d.wait_event(self._computed[k])
+                for i in range(a, b):
+                    self.grads[i].copy_(self.host_grads[i], non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(self.h2d)
+            self.compute.wait_event(arrived)
+            if self._copied_out[k] is not None:
+                self.compute.wait_event(self._copied_out[k])
+            self.steps[k](stream=self.compute)
+            ev = torch.cuda.Event()
+            ev.record(self.compute)
+            self._computed[k] = ev
+            with torch.cuda.stream(self.d2h):
+                self.d2h.wait_event(ev)
+                for i in range(a, b):
+                    self.host_params[i].copy_(self.params[i], non_blocking=True)
+                out = torch.cuda.Event()
+                out.record(self.d2h)
+            self._copied_out[k] = out
+            done.append(out)
+        for ev in done:
+            caller.wait_event(ev)
+
+    @property
+    def status(self) -> torch.Tensor:
+        return torch.cat([st.status_in_param_order() for st in self.steps])
