@@ -27,6 +27,8 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <atomic>
+
 #include "tc_common.cuh"
 
 namespace muon {
@@ -219,14 +221,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn get_encode() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  // thread-safe one-time lookup (the entry point does not depend on the device)
+  static const EncodeTiledFn fn = [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    return static_cast<EncodeTiledFn>(nullptr);
+  }();
   return fn;
 }
 
@@ -254,11 +257,14 @@ bool encode_out_map(CUtensorMap* map, const GemmDesc& g) {
 template <bool B_MN, int IN_FMT, bool SYM>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
                   cudaStream_t s) {
-  static bool attr_done = false;
-  if (!attr_done) {
+  // the shared-memory opt-in is a per-device function attribute: set once per device
+  static std::atomic<int> attr_done[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return (int)cudaErrorInvalidDevice;
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(gemm_kernel<B_MN, IN_FMT, SYM>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return (int)e;
-    attr_done = true;
+    attr_done[dev].store(1, std::memory_order_release);
   }
   const int grid = p.total_tiles < num_sms() ? p.total_tiles : num_sms();
   gemm_kernel<B_MN, IN_FMT, SYM><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, md, p);
@@ -297,11 +303,10 @@ int gemm_tc(const GemmDesc& g, cudaStream_t s) {
 
   // 256-row products go to the paired-CTA kernel (a third less operand
   // traffic per MMA); MUON_GEMM_PAIR=0 keeps every product on the 1-CTA one.
-  static int use_pair = -1;
-  if (use_pair < 0) {
+  static const int use_pair = [] {
     const char* e = getenv("MUON_GEMM_PAIR");
-    use_pair = (e && e[0] == '0') ? 0 : 1;
-  }
+    return (e && e[0] == '0') ? 0 : 1;
+  }();
   if (use_pair && g.M >= 256) return gemm_tc_pair(g, p, s);
 
   CUtensorMap ma, mb;
@@ -323,25 +328,31 @@ int gemm_tc(const GemmDesc& g, cudaStream_t s) {
   return fmt ? launch<false, 1, false>(ma, mb, md, p, s) : launch<false, 0, false>(ma, mb, md, p, s);
 }
 
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
 int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  int n = cached[dev].load(std::memory_order_acquire);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_release);
   }
   return n;
 }
 
 long long wait_timeout_ns() {
-  static long long ns = -1;
-  if (ns < 0) {
+  static const long long ns = [] {
     const char* e = getenv("MUON_WAIT_TIMEOUT_MS");
     long long ms = e ? atoll(e) : 4000;
     if (ms <= 0) ms = 4000;
-    ns = ms * 1000000LL;
-  }
+    return ms * 1000000LL;
+  }();
   return ns;
 }
 

@@ -15,6 +15,8 @@
 // Waits are bounded as in the 1-CTA kernel.
 #include <stdio.h>
 
+#include <atomic>
+
 #include "tc_common.cuh"
 
 namespace muon {
@@ -279,7 +281,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
 template <bool B_MN, int IN_FMT, bool SYM>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
                   cudaStream_t s) {
-  static int max_pairs = 0;
+  // per device: shared-memory opt-in done and how many CTA pairs fit at once
+  static std::atomic<int> max_pairs_of[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return (int)cudaErrorInvalidDevice;
   auto kern = gemm_pair_kernel<B_MN, IN_FMT, SYM>;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
@@ -292,7 +297,8 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMa
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (max_pairs == 0) {
+  int max_pairs = max_pairs_of[dev].load(std::memory_order_acquire);
+  if (max_pairs <= 0) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES2);
     if (e != cudaSuccess) return (int)e;
     cfg.gridDim = dim3(2 * (num_sms() / 2));
@@ -300,6 +306,7 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMa
     e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
     if (e != cudaSuccess || n <= 0) n = num_sms() / 2;
     max_pairs = n;
+    max_pairs_of[dev].store(n, std::memory_order_release);
   }
   const int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   cfg.gridDim = dim3(2 * pairs);

@@ -85,7 +85,10 @@ int gemm_tc(const GemmDesc& g, cudaStream_t s);
 // SIMT path (any dtype, fp32 math): used for fp32 compute.
 int gemm_simt(const GemmDesc& g, cudaStream_t s);
 
-int num_sms();
+// Per-device caches cover device ordinals below kMaxDevices.
+constexpr int kMaxDevices = 64;
+int current_device();   // -1 on error or an ordinal beyond kMaxDevices
+int num_sms();          // of the current device (cached per device)
 long long wait_timeout_ns();
 
 }  // namespace muon
