@@ -322,11 +322,14 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
     if (q_acc < 0) {
       q_acc = qi;
     } else {
-      // Q_acc <- Q Q_acc
+      // Q_acc <- Q Q_acc.  Every Q_k is a polynomial in the same R_0, so the
+      // product is symmetric in exact arithmetic: formed on the upper triangle
+      // and mirrored, like the other symmetric products.
       int ni = 0;
       while (ni == q_acc || ni == qi) ++ni;
       const int n_dt = to_apply ? xdt : gdt;
       sq(g, Qbuf[qi], Qbuf[q_acc], 0, Qbuf[ni], n_dt);
+      g.symmetric = 1;
       if ((rc = gemm(c, g))) return rc;
       q_acc = ni;
     }
