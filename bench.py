@@ -449,7 +449,12 @@ def main():
         host_free = psutil.virtual_memory().available
     except Exception:
         host_free = 0
-    if not args.no_e2e and host_need > 0.6 * host_free:
+    fits = host_need <= 0.6 * host_free
+    if dist is not None:  # every rank must take the same branch (the leg has barriers)
+        flag = torch.tensor([1.0 if fits else 0.0], device=device)
+        dist.all_reduce(flag, op=dist.ReduceOp.MIN)
+        fits = bool(flag.item() > 0.5)
+    if not args.no_e2e and not fits:
         e2e = {"value": None, "unit": "TFLOP/s", "skipped": f"pinned host buffers ({host_need / 2**30:.0f} GiB "
                f"for {local_world} ranks) exceed 60% of free host memory ({host_free / 2**30:.0f} GiB)"}
     elif not args.no_e2e and not args.sharded:
