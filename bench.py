@@ -53,7 +53,7 @@ def parse_args():
     p.add_argument("--workload", choices=["kimi-k2", "kimi-k2-experts16", "dense", "moe", "single"], default="kimi-k2",
                    help="kimi-k2-experts16: 16 expert matrices of the K2 set (small case for profiling)")
     p.add_argument("--mode", choices=["standard", "gram", "gram_stabilized"], default="standard")
-    p.add_argument("--compute", choices=["bf16", "fp16"], default=None,
+    p.add_argument("--compute", choices=["bf16", "fp16", "fp32"], default=None,
                    help="16-bit storage type of the standard chain (default: the workload's, bf16)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
@@ -180,22 +180,39 @@ class ClockSampler:
                 "power_w_max": max(num(r[3]) for r in rows)}
 
 
-def roofline_from_profile(prof, peaks, peak_kind, workload=None):
-    gemm = [r for r in prof if r["kernel"].startswith("tc_product")]
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor rate on B200
+
+
+def roofline_from_profile(prof, peaks, peak_kind, workload=None, compute="bf16"):
+    fp32 = compute == "fp32"
+    gemm = [r for r in prof if r["kernel"].startswith("tc_product") and r["kernel"].endswith("[3xtf32]") == fp32]
     if not gemm:
         return None
     fl = sum(r["flops"] for r in gemm)
     ms = sum(r["ms"] for r in gemm)
     n = sum(r["launches"] for r in gemm)
+    bf16_peak = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
+    if fp32:
+        # three TF32 MMAs per product term (hi*hi, hi*lo, lo*hi): executed TF32 FLOP/s against
+        # the TF32 peak, i.e. the measured BF16 peak times the nominal TF32 : BF16 ratio
+        achieved = 3 * fl / (ms / 1e3) / 1e12
+        peak = round(bf16_peak * TF32_PER_BF16, 1)
+        return {"bound": "tensor",
+                "kernel": "tcgen05 kind::tf32 3xTF32 product kernel (gemm_tf32x3_kernel), all launches of the step",
+                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_kind} bf16_tflops_sustained x {TF32_PER_BF16:.4f} (nominal TF32:BF16), "
+                               "achieved counts the three TF32 MMAs per product term",
+                "algorithmic_tflops": round(fl / (ms / 1e3) / 1e12, 1),
+                "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n,
+                "traffic": None, "traffic_note": "not captured for this kernel"}
     achieved = fl / (ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
     return {"bound": "tensor",
             "kernel": "tcgen05 product kernels (gemm_pair_kernel, gemm_kernel below 256 rows), all launches of the step",
-            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+            "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
             "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
             "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
             "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n,
-            "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get(workload),
+            "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get(workload) if compute == "bf16" else None,
             "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per product launch (ncu, one step)"}
 
 
@@ -353,7 +370,7 @@ def main():
     w, params, grads, moms = build_workload(args.workload, device)
     hp = dict(w.hp, mode=args.mode)
     compute = hp.get("compute_dtype", "bf16")
-    if args.compute is not None and compute != "fp32":
+    if args.compute is not None:
         compute = args.compute
     ws_cap = int(args.workspace_gb * (1 << 30))
     step_hp = dict(lr=hp["lr"], momentum=hp["momentum"], nesterov=hp["nesterov"], weight_decay=hp["weight_decay"],
@@ -489,7 +506,7 @@ def main():
         cpu = cpu_baseline_sample(w, hp)
 
     if rank == 0:
-        roof = roofline_from_profile(prof, peaks, peak_kind, args.workload)
+        roof = roofline_from_profile(prof, peaks, peak_kind, args.workload, compute)
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,

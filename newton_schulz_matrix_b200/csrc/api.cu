@@ -10,6 +10,7 @@
 // R = X X^T, accumulate Q_acc = Q_k ... Q_1, restart once in the stabilised
 // variant) and the optimizer step of "Moonlight 16B Guide" (box steps 1-4).
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -30,10 +31,13 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int round8(int v) { return (v + 7) / 8 * 8; }
 
 // ------------------------------------------------------------------ profiler
-enum ProfKind { kProfPack, kProfNorm, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfKinds };
+enum ProfKind {
+  kProfPack, kProfNorm, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfFusedSmall, kProfTf32, kProfKinds
+};
 // product kinds cover both tensor-core kernels (gemm_pair_kernel for M >= 256, gemm_kernel below)
 const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "tc_product[symmetric]", "tc_product",
-                                            "gemm_simt_kernel", "unpack_kernel"};
+                                            "gemm_simt_kernel", "unpack_kernel", "ns_fused_small_kernel",
+                                            "tc_product[3xtf32]"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -178,15 +182,32 @@ struct Ctx {
   int* err;
 };
 
+// fp32 products with 256 or more rows run as 3xTF32 on the tensor cores;
+// MUON_FP32_TC=0 keeps every fp32 product on the SIMT kernel.
+bool fp32_tensor_cores() {
+  static const bool on = [] {
+    const char* e = getenv("MUON_FP32_TC");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 int gemm(const Ctx& c, GemmDesc g) {
   g.err = c.err;
   const double flops = 2.0 * g.M * g.N * (double)g.K * g.batch;
   const int es = dtype_size(g.in_dtype);
   const double bytes = ((double)g.M * g.K * es + (double)g.N * g.K * es + (double)g.M * g.N * dtype_size(g.d_dtype) +
                         (g.C ? (double)g.M * g.N * dtype_size(g.c_dtype) : 0.0)) * g.batch;
-  const int kind = c.compute == MUON_FP32 ? kProfGemmSimt : (g.symmetric ? kProfSyrkTc : kProfGemmTc);
-  ProfScope ps(kind, flops, bytes, c.s);
-  return c.compute == MUON_FP32 ? gemm_simt(g, c.s) : gemm_tc(g, c.s);
+  if (c.compute == MUON_FP32) {
+    if (g.M >= 256 && fp32_tensor_cores()) {
+      ProfScope ps(kProfTf32, flops, bytes, c.s);
+      return gemm_tf32x3(g, c.s);
+    }
+    ProfScope ps(kProfGemmSimt, flops, bytes, c.s);
+    return gemm_simt(g, c.s);
+  }
+  ProfScope ps(g.symmetric ? kProfSyrkTc : kProfGemmTc, flops, bytes, c.s);
+  return gemm_tc(g, c.s);
 }
 
 GemmDesc desc(int M, int N, int K, int batch) {
@@ -211,8 +232,44 @@ int chain_dtype(const muon_ns_params* ns) {
   return ns->mode == MUON_NS_STANDARD ? ns->compute_dtype : ns->gram_dtype;
 }
 
+// fp32 chains whose matrices fit in one CTA's shared memory run as a single
+// fused launch (one CTA per matrix); MUON_FUSED_SMALL=0 keeps the chained
+// products instead.
+bool fused_small_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("MUON_FUSED_SMALL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+bool use_fused_small(const Layout& L, const muon_ns_params* ns) {
+  if (ns->compute_dtype != MUON_FP32 || ns->iters > FusedSmallArgs::kMaxIters || !fused_small_enabled()) return false;
+  return fused_small_smem(L.n, L.m, ns->mode == MUON_NS_STANDARD ? 0 : 1) <= kFusedSmallMaxSmem;
+}
+
+int run_fused_small(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, bool prescaled) {
+  FusedSmallArgs a{};
+  a.n = L.n; a.m = L.m; a.count = chunk;
+  a.x = reinterpret_cast<float*>(B.X[0]); a.ld_x = L.ld_m; a.x_bs = B.x_bs;
+  a.inv = B.inv; a.raw = prescaled ? 0 : 1;
+  a.mode = ns->mode == MUON_NS_STANDARD ? 0 : 1;
+  a.restart_after = ns->mode == MUON_NS_GRAM_STABILIZED ? ns->restart_after : 0;
+  a.iters = ns->iters;
+  for (int i = 0; i < 3 * ns->iters; ++i) a.coeffs[i] = ns->coeffs[i];
+  const double n = L.n, m = L.m, K = ns->iters;
+  const double flops = a.mode == 0 ? K * (4.0 * m * n * n + 2.0 * n * n * n) : 0.0;
+  ProfScope ps(kProfFusedSmall, flops * chunk, 2.0 * chunk * n * m * 4, c.s);
+  return launch_fused_small(a, c.s);
+}
+
 int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, bool prescaled,
               int* out_x, int* out_dtype) {
+  if (use_fused_small(L, ns)) {
+    *out_x = 0;
+    *out_dtype = MUON_FP32;
+    return run_fused_small(c, L, B, chunk, ns, prescaled);
+  }
   const int n = L.n, m = L.m, K = ns->iters;
   const int cdt = chain_dtype(ns);
   const int xdt = cdt;  // X storage

@@ -2,6 +2,8 @@
 // kernel.  It carries the fp32 compute mode: tcgen05 offers only TF32 for
 // 32-bit operands, whose 10-bit mantissa cannot hold a 1e-4 relative error
 // through five Newton-Schulz iterations.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -95,6 +97,167 @@ int gemm_simt(const GemmDesc& g, cudaStream_t s) {
     case kFP16: gemm_simt_kernel<__half><<<grid, 256, 0, s>>>(g); break;
     default: gemm_simt_kernel<float><<<grid, 256, 0, s>>>(g); break;
   }
+  return (int)cudaGetLastError();
+}
+
+
+
+
+// ----------------------------------------------------------------------------
+// Fused fp32 chain for small matrices: one CTA per matrix runs every product of
+// the iteration in shared memory, so the whole Newton-Schulz chain is a single
+// launch.  The products are the same as the chained kernels' (standard form:
+// A = X X^T, B = b A + c A A, X <- a X + B X; Gram form: R = X X^T,
+// Q = a I + b R + c R R, Q_acc <- Q Q_acc, R <- (Q R) Q, restart, X = Q_acc X0),
+// here with plain R R (no symmetric shortcut is needed in shared memory).
+// ----------------------------------------------------------------------------
+namespace {
+
+constexpr int kFusedThreads = 256;
+
+// C = alpha * A op(B) + beta * Cin + eye * I, all in shared memory.
+// A: M x K (lda).  NT: B stored N x K (C = A B^T), else K x N (C = A B).
+// 16 x 16 threads, each a 4 x 4 block of a 64 x 64 output tile.  Rows and
+// columns past M / N read a clamped (valid) index and are not stored, so the
+// k loop carries no predicates.
+template <bool NT>
+__device__ void smem_mm(const float* A, int lda, const float* B, int ldb, float* C, int ldc, int M, int N, int K,
+                        float alpha, const float* Cin, int ldcin, float beta, float eye) {
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  for (int i0 = 0; i0 < M; i0 += 64) {
+    for (int j0 = 0; j0 < N; j0 += 64) {
+      const float* ap[4];
+      const float* bp[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) ap[r] = A + min(i0 + ty + 16 * r, M - 1) * lda;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = min(j0 + tx + 16 * c, N - 1);
+        bp[c] = NT ? B + j * ldb : B + j;
+      }
+      float acc[4][4] = {};
+#pragma unroll 4
+      for (int k = 0; k < K; ++k) {
+        float av[4], bv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) av[r] = ap[r][k];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) bv[c] = NT ? bp[c][k] : bp[c][k * ldb];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(av[r], bv[c], acc[r][c]);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = i0 + ty + 16 * r;
+        if (i >= M) continue;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int j = j0 + tx + 16 * c;
+          if (j >= N) continue;
+          float v = alpha * acc[r][c];
+          if (Cin) v += beta * Cin[i * ldcin + j];
+          if (i == j) v += eye;
+          C[i * ldc + j] = v;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
+__device__ void smem_identity(float* Q, int ld, int n) {
+  for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
+    const int i = e / n, j = e % n;
+    Q[i * ld + j] = i == j ? 1.f : 0.f;
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kFusedThreads)
+ns_fused_small_kernel(const FusedSmallArgs a) {
+  extern __shared__ float sm[];
+  const int n = a.n, m = a.m, ldx = m + 1, ldn = n + 1;  // odd strides: conflict-free columns
+  float* X = sm;
+  float* Y = X + n * ldx;
+  float* S = Y + n * ldx;  // Gram-sized matrices, ldn each
+  float* xg = a.x + (long long)blockIdx.x * a.x_bs;
+  const float f = a.raw ? a.inv[blockIdx.x] : 1.f;
+  for (int e = threadIdx.x; e < n * m; e += blockDim.x) {
+    const int i = e / m, j = e % m;
+    X[i * ldx + j] = f * xg[(long long)i * a.ld_x + j];
+  }
+  __syncthreads();
+  if (a.mode == 0) {
+    float* Am = S;
+    float* Bm = S + n * ldn;
+    for (int k = 0; k < a.iters; ++k) {
+      const float ca = a.coeffs[3 * k], cb = a.coeffs[3 * k + 1], cc = a.coeffs[3 * k + 2];
+      smem_mm<true>(X, ldx, X, ldx, Am, ldn, n, n, m, 1.f, nullptr, 0, 0.f, 0.f);       // A = X X^T
+      const float* P = Am;
+      float coef = cb;
+      if (cc != 0.f) {
+        smem_mm<false>(Am, ldn, Am, ldn, Bm, ldn, n, n, n, cc, Am, ldn, cb, 0.f);       // B = c A A + b A
+        P = Bm;
+        coef = 1.f;
+      }
+      smem_mm<false>(P, ldn, X, ldx, Y, ldx, n, m, n, coef, X, ldx, ca, 0.f);           // X' = a X + B X
+      float* t = X; X = Y; Y = t;
+    }
+  } else {
+    float* R = S;
+    float* Q = R + n * ldn;
+    float* T = Q + n * ldn;
+    float* Qa = T + n * ldn;
+    float* Qb = Qa + n * ldn;
+    smem_mm<true>(X, ldx, X, ldx, R, ldn, n, n, m, 1.f, nullptr, 0, 0.f, 0.f);         // R = X0 X0^T
+    smem_identity(Qa, ldn, n);
+    for (int k = 1; k <= a.iters; ++k) {
+      const float ca = a.coeffs[3 * (k - 1)], cb = a.coeffs[3 * (k - 1) + 1], cc = a.coeffs[3 * (k - 1) + 2];
+      smem_mm<false>(R, ldn, R, ldn, Q, ldn, n, n, n, cc, R, ldn, cb, ca);              // Q = a I + b R + c R R
+      smem_mm<false>(Q, ldn, Qa, ldn, Qb, ldn, n, n, n, 1.f, nullptr, 0, 0.f, 0.f);      // Q_acc <- Q Q_acc
+      float* t = Qa; Qa = Qb; Qb = t;
+      if (k == a.iters) break;
+      if (a.restart_after > 0 && k == a.restart_after) {
+        smem_mm<false>(Qa, ldn, X, ldx, Y, ldx, n, m, n, 1.f, nullptr, 0, 0.f, 0.f);     // X <- Q_acc X0
+        float* u = X; X = Y; Y = u;
+        smem_mm<true>(X, ldx, X, ldx, R, ldn, n, n, m, 1.f, nullptr, 0, 0.f, 0.f);       // R <- X X^T
+        smem_identity(Qa, ldn, n);
+      } else {
+        smem_mm<false>(Q, ldn, R, ldn, T, ldn, n, n, n, 1.f, nullptr, 0, 0.f, 0.f);      // T = Q R
+        smem_mm<false>(T, ldn, Q, ldn, R, ldn, n, n, n, 1.f, nullptr, 0, 0.f, 0.f);      // R <- T Q
+      }
+    }
+    smem_mm<false>(Qa, ldn, X, ldx, Y, ldx, n, m, n, 1.f, nullptr, 0, 0.f, 0.f);         // X = Q_acc X0
+    X = Y;
+  }
+  for (int e = threadIdx.x; e < n * m; e += blockDim.x) {
+    const int i = e / m, j = e % m;
+    xg[(long long)i * a.ld_x + j] = X[i * ldx + j];
+  }
+}
+
+size_t fused_small_smem(int n, int m, int mode) {
+  const size_t sq = mode == 0 ? 2 : 5;
+  return sizeof(float) * (2 * (size_t)n * (m + 1) + sq * (size_t)n * (n + 1));
+}
+
+int launch_fused_small(const FusedSmallArgs& a, cudaStream_t s) {
+  const size_t bytes = fused_small_smem(a.n, a.m, a.mode);
+  if (bytes > kFusedSmallMaxSmem || a.iters > FusedSmallArgs::kMaxIters) return (int)cudaErrorInvalidValue;
+  static std::atomic<int> attr_done[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return (int)cudaErrorInvalidDevice;
+  if (!attr_done[dev].load(std::memory_order_acquire)) {
+    cudaError_t e = cudaFuncSetAttribute(ns_fused_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kFusedSmallMaxSmem);
+    if (e != cudaSuccess) return (int)e;
+    attr_done[dev].store(1, std::memory_order_release);
+  }
+  ns_fused_small_kernel<<<a.count, kFusedThreads, bytes, s>>>(a);
   return (int)cudaGetLastError();
 }
 

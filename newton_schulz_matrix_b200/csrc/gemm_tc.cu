@@ -235,15 +235,20 @@ static EncodeTiledFn get_encode() {
 
 // 3-D tiled map over a batch of row-major matrices: dims (inner, outer, batch).
 bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer, long long batch,
-                long long ld_elems, long long bs_elems, int box_inner, int box_outer, int swizzle_bytes) {
+                long long ld_elems, long long bs_elems, int box_inner, int box_outer, TmaSwizzle swizzle) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
-  const CUtensorMapDataType dt = dtype == kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType dt = dtype == kBF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                 : dtype == kFP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                  : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const long long es = dtype_size(dtype);
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)outer, (cuuint64_t)batch};
-  cuuint64_t strides[2] = {(cuuint64_t)ld_elems * 2, (cuuint64_t)(bs_elems > 0 ? bs_elems : ld_elems * outer) * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)(ld_elems * es), (cuuint64_t)((bs_elems > 0 ? bs_elems : ld_elems * outer) * es)};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  const CUtensorMapSwizzle sw = swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUtensorMapSwizzle sw = swizzle == kTmaSw64          ? CU_TENSOR_MAP_SWIZZLE_64B
+                                : swizzle == kTmaSw128Atom32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                                             : CU_TENSOR_MAP_SWIZZLE_128B;
   CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -251,7 +256,7 @@ bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, 
 }
 
 bool encode_out_map(CUtensorMap* map, const GemmDesc& g) {
-  return encode_map(map, g.d_dtype, g.D, g.N, g.M, g.batch, g.ldd, g.d_bs, 32, 32, 64);
+  return encode_map(map, g.d_dtype, g.D, g.N, g.M, g.batch, g.ldd, g.d_bs, 32, 32, kTmaSw64);
 }
 
 template <bool B_MN, int IN_FMT, bool SYM>

@@ -29,20 +29,6 @@ constexpr int B_BYTES2 = 128 * BK * 2;  // this CTA's 128 columns of B: 16 KB
 constexpr int STAGE_BYTES2 = A_BYTES2 + B_BYTES2;
 constexpr int SMEM_BYTES2 = STAGES2 * STAGE_BYTES2 + STAGING_BYTES + 1024 + 256;
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// Address of the same shared-memory object in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y, int z) {
   asm volatile(
@@ -60,45 +46,6 @@ __device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Arrive (once MMAs issued so far retire) on the barrier at this offset in
-// every CTA of `mask`.
-__device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
-      "h"(mask)
-      : "memory");
-}
-__device__ __forceinline__ void remote_arrive(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
-}
-
-struct PairTile { int b, TM, TN; };
-
-__device__ __forceinline__ PairTile decode_pair(const Params& p, int t) {
-  PairTile r;
-  r.b = t / p.tiles_per_batch;
-  int q = t - r.b * p.tiles_per_batch;
-  if (p.symmetric) {
-    int tm = 0;
-    for (; tm < p.tiles_m; ++tm) {
-      const int cnt = p.tiles_n - tm;
-      if (q < cnt) break;
-      q -= cnt;
-    }
-    r.TM = tm;
-    r.TN = tm + q;
-  } else {
-    const int per_group = GROUP_M * p.tiles_n;
-    const int g = q / per_group;
-    const int first = g * GROUP_M;
-    const int gsz = min(p.tiles_m - first, GROUP_M);
-    const int w = q - g * per_group;
-    r.TM = first + w % gsz;
-    r.TN = w / gsz;
-  }
-  return r;
-}
-
 template <bool B_MN, int IN_FMT, bool SYM>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,

@@ -82,8 +82,27 @@ struct GemmDesc {
 };
 // Tensor-core (tcgen05) path: bf16/fp16 operands.  Returns 0 or a CUDA error.
 int gemm_tc(const GemmDesc& g, cudaStream_t s);
-// SIMT path (any dtype, fp32 math): used for fp32 compute.
+// Tensor-core path for fp32 operands (3xTF32, paired CTAs): fp32 A, B, C and D.
+int gemm_tf32x3(const GemmDesc& g, cudaStream_t s);
+// SIMT path (any dtype, fp32 math): fp32 products with fewer than 256 rows.
 int gemm_simt(const GemmDesc& g, cudaStream_t s);
+
+// Whole fp32 Newton-Schulz chain of small matrices, one CTA per matrix, in
+// shared memory (single launch).  x: workspace batch (count x n x ld_x fp32),
+// overwritten with the result; raw: scale by inv[b] on load.
+struct FusedSmallArgs {
+  static constexpr int kMaxIters = 64;
+  int n, m, count;
+  float* x; int ld_x; long long x_bs;
+  const float* inv; int raw;
+  int mode;            // 0 standard, 1 Gram (restart_after 0 = naive)
+  int restart_after;
+  int iters;
+  float coeffs[3 * kMaxIters];
+};
+constexpr size_t kFusedSmallMaxSmem = 200 * 1024;
+size_t fused_small_smem(int n, int m, int mode);
+int launch_fused_small(const FusedSmallArgs& a, cudaStream_t s);
 
 // Per-device caches cover device ordinals below kMaxDevices.
 constexpr int kMaxDevices = 64;

@@ -129,14 +129,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor, sm_100 version field.  Layout 2 is the
+// 128-byte swizzle with 16-byte granules (every K-major operand, and 16-bit
+// MN-major ones); layout 1 is the 128-byte swizzle with 32-byte granules,
+// which 32-bit (TF32) MN-major operands take.
+constexpr uint32_t kLayoutSw128 = 2;
+constexpr uint32_t kLayoutSw128Atom32 = 1;
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout = kLayoutSw128) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
-  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  d |= (uint64_t)layout << 61;
   return d;
 }
 
@@ -318,10 +324,69 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMa
   }
 }
 
+// ------------------------------------------------------------------ clusters of two CTAs
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive (once MMAs issued so far retire) on the barrier at this offset in
+// every CTA of `mask`.
+__device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void remote_arrive(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+// Tile order of the paired-CTA kernels: 256 x 256 tiles (upper triangle only
+// for symmetric products), grouped rasterisation otherwise.
+struct PairTile { int b, TM, TN; };
+
+__device__ __forceinline__ PairTile decode_pair(const Params& p, int t) {
+  PairTile r;
+  r.b = t / p.tiles_per_batch;
+  int q = t - r.b * p.tiles_per_batch;
+  if (p.symmetric) {
+    int tm = 0;
+    for (; tm < p.tiles_m; ++tm) {
+      const int cnt = p.tiles_n - tm;
+      if (q < cnt) break;
+      q -= cnt;
+    }
+    r.TM = tm;
+    r.TN = tm + q;
+  } else {
+    const int per_group = GROUP_M * p.tiles_n;
+    const int g = q / per_group;
+    const int first = g * GROUP_M;
+    const int gsz = min(p.tiles_m - first, GROUP_M);
+    const int w = q - g * per_group;
+    r.TM = first + w % gsz;
+    r.TN = w / gsz;
+  }
+  return r;
+}
+
 // ------------------------------------------------------------------ host side (gemm_tc.cu)
-// 3-D tiled tensor map over a batch of row-major matrices, 128-byte swizzle.
+// 3-D tiled tensor map over a batch of row-major matrices.  Shared-memory
+// layouts: 128-byte swizzle (16-byte granules), 64-byte swizzle, or 128-byte
+// swizzle with 32-byte granules (TF32 MN-major operands).
+enum TmaSwizzle { kTmaSw128, kTmaSw64, kTmaSw128Atom32 };
 bool encode_map(CUtensorMap* map, int dtype, const void* base, long long inner, long long outer, long long batch,
-                long long ld_elems, long long bs_elems, int box_inner, int box_outer, int swizzle_bytes = 128);
+                long long ld_elems, long long bs_elems, int box_inner, int box_outer, TmaSwizzle swizzle = kTmaSw128);
 // Output map of a product: 32 x 32 boxes, 64-byte swizzle (the epilogue's staging layout).
 bool encode_out_map(CUtensorMap* map, const GemmDesc& g);
 // 2-CTA (cta_group::2) variant for 256-row tiles (gemm_tc2.cu).

@@ -142,6 +142,73 @@ def test_fp32_cubic_40_steps_is_polar_factor():
 
 
 # ---------------------------------------------------------------------------
+# fp32 chains of small matrices run as one fused launch (one CTA per matrix,
+# the whole chain in shared memory): ragged sizes below and across the 16 x 16
+# thread grid and the 64 x 64 output tile, batches wider than the SM count, and
+# a schedule longer than the fused kernel's coefficient table (chained products)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(37, 53), (17, 200), (100, 64), (64, 65), (90, 91)])
+@pytest.mark.parametrize("mode", ["standard", "gram", "gram_stabilized"])
+def test_fp32_small_matrix_chain(shape, mode):
+    mats = [synth.gaussian(*shape, seed=500 + i + shape[0], device=DEV) for i in range(3)]
+    ys, st = gpu_ns(mats, mode=mode, compute_dtype="fp32")
+    assert st == [0, 0, 0]
+    for x, y in zip(mats, ys):
+        U = to_np(x)
+        assert rel(to_np(y), oracle.newton_schulz(U, Q5, mode=mode)) < 1e-4
+
+
+def test_fp32_small_matrix_chain_wide_batch_and_long_schedule():
+    mats = [synth.gaussian(48, 96, seed=900 + i, device=DEV) for i in range(300)]
+    ys, st = gpu_ns(mats, compute_dtype="fp32")
+    assert st == [0] * 300
+    for i in (0, 147, 148, 299):
+        assert rel(to_np(ys[i]), oracle.newton_schulz(to_np(mats[i]), Q5)) < 1e-4
+    coeffs = [oracle.CUBIC] * 70
+    (y,), st = gpu_ns(mats[:1], coeffs=coeffs, compute_dtype="fp32")
+    assert st == [0]
+    assert rel(to_np(y), oracle.newton_schulz(to_np(mats[0]), coeffs)) < 1e-4
+
+
+# ---------------------------------------------------------------------------
+# fp32 chains with n >= 256 run on the tensor cores as 3xTF32 (hi/lo split of
+# every operand): ragged 256-tiles, tall and wide, all three forms at the fp32
+# bar; symmetric products come out exactly symmetric (mirrored upper triangle)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape", [(300, 700), (520, 260), (640, 640), (256, 2056)])
+@pytest.mark.parametrize("mode", ["standard", "gram", "gram_stabilized"])
+def test_fp32_tensor_core_chain(shape, mode):
+    mats = [synth.gaussian(*shape, seed=700 + i + shape[0], device=DEV) for i in range(2)]
+    ys, st = gpu_ns(mats, mode=mode, compute_dtype="fp32")
+    assert st == [0, 0]
+    for x, y in zip(mats, ys):
+        U = to_np(x)
+        assert rel(to_np(y), oracle.newton_schulz(U, Q5, mode=mode)) < 1e-4
+
+
+@pytest.mark.parametrize("abc", [(0.0, 1.0, 0.0), (0.0, 0.0, 1.0)])
+def test_fp32_tensor_core_single_products(abc):
+    """One iteration isolates X X^T X (b) and (X X^T)^2 X (c) on the 3xTF32 path."""
+    X = synth.gaussian(300, 777, seed=31, device=DEV)
+    (Y,), st = gpu_ns([X], coeffs=[abc], compute_dtype="fp32")
+    assert st == [0]
+    assert rel(to_np(Y), oracle.newton_schulz(to_np(X), [abc])) < 1e-5  # one TF32 pass: ~5e-4
+
+
+@pytest.mark.parametrize("mode", ["standard", "gram", "gram_stabilized"])
+def test_fp32_dense_projection_shape(mode):
+    """1024 x 4096 (the dense-projection shape): K = 4096 in X X^T, where an
+    unfolded tensor-core accumulation would leave the fp32 bar."""
+    mats = [synth.low_rank_plus_noise(1024, 4096, 64, 0.1, seed=810 + i, device=DEV) for i in range(2)]
+    ys, st = gpu_ns(mats, mode=mode, compute_dtype="fp32")
+    assert st == [0, 0]
+    U = to_np(mats[0])
+    y = to_np(ys[0])
+    assert rel(y, oracle.newton_schulz(U, Q5, mode=mode)) < 1e-4
+    assert sigma_band_error(U, y, Q5) < 0.05
+
+
+# ---------------------------------------------------------------------------
 # Muon step: momentum, Nesterov, orientation merge, decay and scale
 # ---------------------------------------------------------------------------
 def _groups_for_step(spec, w_dtype, seed):
