@@ -117,32 +117,72 @@ constexpr int kFusedThreads = 256;
 
 // C = alpha * A op(B) + beta * Cin + eye * I, all in shared memory.
 // A: M x K (lda).  NT: B stored N x K (C = A B^T), else K x N (C = A B).
-// 16 x 16 threads, each a 4 x 4 block of a 64 x 64 output tile.  Rows and
-// columns past M / N read a clamped (valid) index and are not stored, so the
-// k loop carries no predicates.
+// 16 x 16 threads, each a 4 x 4 block of a 64 x 64 output tile: rows
+// i0 + ty + 16 r; columns j0 + tx + 16 c (NT) or j0 + 4 tx + c (NN, so that a
+// thread's four B values are one 16-byte load).  k advances by 4 with 16-byte
+// loads (a warp's A rows are two broadcast addresses; its B reads are 256
+// contiguous or row-strided bytes), then a scalar tail.  Every leading
+// dimension is a multiple of 4 whose quarter is odd, which keeps 16-byte loads
+// aligned and row-strided ones free of bank conflicts.  Rows and columns past
+// M / N read a clamped (valid) index and are not stored, so the k loop carries
+// no predicates.
 template <bool NT>
 __device__ void smem_mm(const float* A, int lda, const float* B, int ldb, float* C, int ldc, int M, int N, int K,
                         float alpha, const float* Cin, int ldcin, float beta, float eye) {
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int K4 = K & ~3;
   for (int i0 = 0; i0 < M; i0 += 64) {
     for (int j0 = 0; j0 < N; j0 += 64) {
       const float* ap[4];
       const float* bp[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) ap[r] = A + min(i0 + ty + 16 * r, M - 1) * lda;
+      if (NT) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int j = min(j0 + tx + 16 * c, N - 1);
-        bp[c] = NT ? B + j * ldb : B + j;
+        for (int c = 0; c < 4; ++c) bp[c] = B + min(j0 + tx + 16 * c, N - 1) * ldb;
+      } else {
+        bp[0] = B + min(j0 + 4 * tx, (N - 1) & ~3);  // 4 aligned columns inside the row
       }
       float acc[4][4] = {};
-#pragma unroll 4
-      for (int k = 0; k < K; ++k) {
+#pragma unroll 2
+      for (int k = 0; k < K4; k += 4) {
+        float4 av[4], bv[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) av[r] = *reinterpret_cast<const float4*>(ap[r] + k);
+        if (NT) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) bv[c] = *reinterpret_cast<const float4*>(bp[c] + k);
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              acc[r][c] = fmaf(av[r].x, bv[c].x, acc[r][c]);
+              acc[r][c] = fmaf(av[r].y, bv[c].y, acc[r][c]);
+              acc[r][c] = fmaf(av[r].z, bv[c].z, acc[r][c]);
+              acc[r][c] = fmaf(av[r].w, bv[c].w, acc[r][c]);
+            }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) bv[q] = *reinterpret_cast<const float4*>(bp[0] + (k + q) * ldb);
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const float a4[4] = {av[r].x, av[r].y, av[r].z, av[r].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              acc[r][0] = fmaf(a4[q], bv[q].x, acc[r][0]);
+              acc[r][1] = fmaf(a4[q], bv[q].y, acc[r][1]);
+              acc[r][2] = fmaf(a4[q], bv[q].z, acc[r][2]);
+              acc[r][3] = fmaf(a4[q], bv[q].w, acc[r][3]);
+            }
+          }
+        }
+      }
+      for (int k = K4; k < K; ++k) {
         float av[4], bv[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) av[r] = ap[r][k];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) bv[c] = NT ? bp[c][k] : bp[c][k * ldb];
+        for (int c = 0; c < 4; ++c) bv[c] = NT ? bp[c][k] : bp[0][k * ldb + c];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -154,7 +194,7 @@ __device__ void smem_mm(const float* A, int lda, const float* B, int ldb, float*
         if (i >= M) continue;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int j = j0 + tx + 16 * c;
+          const int j = NT ? j0 + tx + 16 * c : j0 + 4 * tx + c;
           if (j >= N) continue;
           float v = alpha * acc[r][c];
           if (Cin) v += beta * Cin[i * ldcin + j];
@@ -165,6 +205,12 @@ __device__ void smem_mm(const float* A, int lda, const float* B, int ldb, float*
     }
   }
   __syncthreads();
+}
+
+// Leading dimension for a row of `cols` floats: a multiple of 4 with an odd quarter.
+__host__ __device__ inline int fused_ld(int cols) {
+  const int q = (cols + 3) / 4;
+  return 4 * (q | 1);
 }
 
 __device__ void smem_identity(float* Q, int ld, int n) {
@@ -180,7 +226,7 @@ __device__ void smem_identity(float* Q, int ld, int n) {
 __global__ void __launch_bounds__(kFusedThreads)
 ns_fused_small_kernel(const FusedSmallArgs a) {
   extern __shared__ float sm[];
-  const int n = a.n, m = a.m, ldx = m + 1, ldn = n + 1;  // odd strides: conflict-free columns
+  const int n = a.n, m = a.m, ldx = fused_ld(m), ldn = fused_ld(n);
   float* X = sm;
   float* Y = X + n * ldx;
   float* S = Y + n * ldx;  // Gram-sized matrices, ldn each
@@ -242,7 +288,7 @@ ns_fused_small_kernel(const FusedSmallArgs a) {
 
 size_t fused_small_smem(int n, int m, int mode) {
   const size_t sq = mode == 0 ? 2 : 5;
-  return sizeof(float) * (2 * (size_t)n * (m + 1) + sq * (size_t)n * (n + 1));
+  return sizeof(float) * (2 * (size_t)n * fused_ld(m) + sq * (size_t)n * fused_ld(n));
 }
 
 int launch_fused_small(const FusedSmallArgs& a, cudaStream_t s) {
