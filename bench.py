@@ -4,7 +4,8 @@ normalisation, five quintic Newton-Schulz iterations, update scaling and
 decoupled weight decay) over the Kimi-K2-shaped parameter set on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload kimi-k2|dense|moe|single] [--mode standard|gram|gram_stabilized]
+                    [--workload kimi-k2|dense|dense16|moe|single] [--mode standard|gram|gram_stabilized]
+                    [--compute bf16|fp16|fp32]
 
 A step is one muon_step call over all matrices of the workload (inputs resident
 in HBM).  The metric is effective TFLOP/s: the iteration's algorithmic FLOPs
@@ -36,11 +37,15 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "NS-orthogonalization ms/optimizer-step & effective TFLOP/s (% of bf16 peak)"
-# DRAM bytes (read + write) per product-kernel launch, averaged over the 45
-# launches of one Kimi-K2 step, from the ncu launch list summarised in
-# profiles/launches_kimi_k2_step.md.  Reset to None whenever the product
-# kernels change until a new capture is taken.
-PRODUCT_TRAFFIC_PER_LAUNCH = {"kimi-k2": 20.79e9}
+# DRAM bytes (read + write) per product-kernel launch, keyed by (workload,
+# compute type).  bf16 Kimi-K2: averaged over the 45 launches of one step
+# (profiles/launches_kimi_k2_step.md).  fp32 dense: the three products of one
+# iteration captured on the 16-matrix set (profiles/gemm_tf32x3_kernel_dense16_fp32.md),
+# averaged (a step repeats them five times), and x4 for the 64-matrix set, whose
+# traffic grows with the matrix count.  Reset an entry to None whenever its
+# kernel changes until a new capture is taken.
+PRODUCT_TRAFFIC_PER_LAUNCH = {("kimi-k2", "bf16"): 20.79e9,
+                              ("dense16", "fp32"): 324.7e6, ("dense", "fp32"): 4 * 324.7e6}
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
@@ -50,11 +55,11 @@ def parse_args():
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", choices=["kimi-k2", "kimi-k2-experts16", "dense", "moe", "single"], default="kimi-k2",
-                   help="kimi-k2-experts16: 16 expert matrices of the K2 set (small case for profiling)")
+    p.add_argument("--workload", choices=["kimi-k2", "kimi-k2-experts16", "dense", "dense16", "moe", "single"], default="kimi-k2",
+                   help="kimi-k2-experts16 / dense16: 16 matrices of the K2 / dense set (small cases for profiling)")
     p.add_argument("--mode", choices=["standard", "gram", "gram_stabilized"], default="standard")
     p.add_argument("--compute", choices=["bf16", "fp16", "fp32"], default=None,
-                   help="16-bit storage type of the standard chain (default: the workload's, bf16)")
+                   help="storage type of the chain (default: the workload's, bf16); fp32 runs 3xTF32 products")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -100,6 +105,8 @@ def build_workload(name, device):
         w = synth.kimi_k2(device=device, counts=[16, 0, 0, 0])
     elif name == "dense":
         w = synth.dense_projection(device=device)
+    elif name == "dense16":  # 16 of the dense matrices: small enough for a full profiler capture
+        w = synth.dense_projection(device=device, count=16)
     elif name == "moe":
         w = synth.moe_layer(device=device)
     else:
@@ -194,17 +201,19 @@ def roofline_from_profile(prof, peaks, peak_kind, workload=None, compute="bf16")
     bf16_peak = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
     if fp32:
         # three TF32 MMAs per product term (hi*hi, hi*lo, lo*hi): executed TF32 FLOP/s against
-        # the TF32 peak, i.e. the measured BF16 peak times the nominal TF32 : BF16 ratio
+        # the TF32 peak, i.e. the measured burst BF16 peak times the nominal TF32 : BF16 ratio
+        # (the fp32 steps run far below the power cap, at the maximum SM clock)
         achieved = 3 * fl / (ms / 1e3) / 1e12
-        peak = round(bf16_peak * TF32_PER_BF16, 1)
+        peak = round(peaks["bf16_tflops"] * TF32_PER_BF16, 1)
         return {"bound": "tensor",
                 "kernel": "tcgen05 kind::tf32 3xTF32 product kernel (gemm_tf32x3_kernel), all launches of the step",
                 "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{peak_kind} bf16_tflops_sustained x {TF32_PER_BF16:.4f} (nominal TF32:BF16), "
+                "peak_source": f"{peak_kind} bf16_tflops (burst) x {TF32_PER_BF16:.4f} (nominal TF32:BF16), "
                                "achieved counts the three TF32 MMAs per product term",
                 "algorithmic_tflops": round(fl / (ms / 1e3) / 1e12, 1),
                 "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n,
-                "traffic": None, "traffic_note": "not captured for this kernel"}
+                "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get((workload, compute)),
+                "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per product launch (ncu)"}
     achieved = fl / (ms / 1e3) / 1e12
     return {"bound": "tensor",
             "kernel": "tcgen05 product kernels (gemm_pair_kernel, gemm_kernel below 256 rows), all launches of the step",
@@ -212,7 +221,7 @@ def roofline_from_profile(prof, peaks, peak_kind, workload=None, compute="bf16")
             "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
             "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
             "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n,
-            "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get(workload) if compute == "bf16" else None,
+            "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get((workload, compute)),
             "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per product launch (ncu, one step)"}
 
 
