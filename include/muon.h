@@ -75,8 +75,11 @@ enum {
  *   eps            X0 = U / (||U||_F + eps)  [Moonlight, NS section; listing eps]
  *   compute_dtype  MUON_BF16 or MUON_FP16: tcgen05 tensor cores, fp32
  *                  accumulate, 16-bit storage of X, A, B between the products
- *                  of the standard form; MUON_FP32: CUDA-core FFMA products in
- *                  fp32 throughout (any mode)
+ *                  of the standard form; MUON_FP32: fp32 storage throughout
+ *                  (any mode), products as 3xTF32 on the tensor cores (operands
+ *                  split into TF32 hi + lo, fp32 sums per 32-deep k-block) when
+ *                  min(rows, cols) >= 256, else fp32 FFMA (a matrix whose whole
+ *                  chain fits in one block's shared memory runs it in one launch)
  *   gram_dtype     Gram modes on tensor cores: the 16-bit type of every matrix
  *                  the Gram chain stores (R, Q, Q_acc, X0 and the restart X),
  *                  MUON_FP16 (the stabilised variant's float16) or MUON_BF16 */
