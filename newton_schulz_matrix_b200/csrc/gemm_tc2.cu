@@ -11,7 +11,10 @@
 //     each), and releases each stage in both CTAs with a multicast commit;
 //   - each CTA drains its own 128 x 256 accumulator (two TMEM buffers) with
 //     the shared epilogue; both CTAs' epilogue warps hand the buffer back to
-//     the leader's MMA issuer through a remote mbarrier arrive.
+//     the leader's MMA issuer through a remote mbarrier arrive;
+//   - a ragged last column tile with at most 128 valid columns (e.g. 1408 =
+//     5.5 x 256) runs N = 128 MMAs, each CTA supplying 64 columns, which halves
+//     its tensor work; its accumulator's upper 128 columns are never stored.
 // Waits are bounded as in the 1-CTA kernel.
 #include <stdio.h>
 
@@ -110,8 +113,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       bool ok = true;
       for (int t = pair; t < p.total_tiles && ok; t += npairs) {
         const PairTile tl = decode_pair(p, t);
-        const int row0 = tl.TM * 256 + (int)rank * 128;   // this CTA's rows of A
-        const int col0 = tl.TN * 256 + (int)rank * 128;   // this CTA's columns of B
+        // a ragged last column tile with at most 128 valid columns runs N = 128
+        // MMAs: each CTA then supplies 64 columns (the first 64 it loads)
+        const bool narrow = p.N - tl.TN * 256 <= 128;
+        const int row0 = tl.TM * 256 + (int)rank * 128;                   // this CTA's rows of A
+        const int col0 = tl.TN * 256 + (int)rank * (narrow ? 64 : 128);  // this CTA's columns of B
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
           if (leader) mbar_expect_tx(smem_u32(&full_bar[stage]), 2 * STAGE_BYTES2);
@@ -134,12 +140,14 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (leader only)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = make_idesc(IN_FMT, B_MN ? 1 : 0, 256);
+      constexpr uint32_t idesc_full = make_idesc(IN_FMT, B_MN ? 1 : 0, 256, 256);
+      constexpr uint32_t idesc_narrow = make_idesc(IN_FMT, B_MN ? 1 : 0, 256, 128);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
       for (int t = pair; t < p.total_tiles && ok; t += npairs, ++it) {
+        const uint32_t idesc = p.N - decode_pair(p, t).TN * 256 <= 128 ? idesc_narrow : idesc_full;
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait(smem_u32(&tempty_bar[acc]), aph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }

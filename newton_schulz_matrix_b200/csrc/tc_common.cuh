@@ -147,10 +147,10 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 }
 
 // Instruction descriptor for kind::f16: fp32 D, A/B of one 16-bit type,
-// A K-major, B K-major or MN-major, M = 128, N = 256.
-__host__ __device__ constexpr uint32_t make_idesc(int in_fmt /*0 f16, 1 bf16*/, int b_mn, int m = BM) {
+// A K-major, B K-major or MN-major, M x N (default 128 x 256).
+__host__ __device__ constexpr uint32_t make_idesc(int in_fmt /*0 f16, 1 bf16*/, int b_mn, int m = BM, int n = BN) {
   return (1u << 4) | ((uint32_t)in_fmt << 7) | ((uint32_t)in_fmt << 10) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
 // ------------------------------------------------------------------ tile order
