@@ -17,11 +17,11 @@
 // Layout: persistent CTA pairs on 256 x 128 output tiles (each CTA 128 rows;
 // the leader issues M=256, N=128, K=8 MMAs reading both CTAs' shared memory).
 //   - each CTA's TMA loads (24 KB of fp32 per k-block) complete on its own
-//     barrier; a converter warpgroup in each CTA then writes hi over the landed
+//     barrier; four converter warps in each CTA then write hi over the landed
 //     tile and lo into a second buffer of the same swizzled layout (the split
-//     is elementwise, so the layout carries over), fences the writes for the
-//     tensor core and arrives on the leader's barrier, which the MMA issuer
-//     waits on;
+//     is elementwise, so the layout carries over), each on its own quarter of
+//     the stage; each warp fences its writes for the tensor core and arrives
+//     on the leader's barrier, which the MMA issuer waits on;
 //   - MN-major B tiles use the 128-byte swizzle with 32-byte granules (the
 //     only shared-memory layout the tensor core takes for 32-bit MN-major
 //     operands), in the tensor map and in the descriptor alike;
@@ -57,7 +57,7 @@ constexpr int NUM_THREADS3 = 64 + 32 * (NUM_EPI_WARPS + NUM_CONV_WARPS);
 constexpr int NUM_BARS3 = 3 * STAGES3 + 2 * NUM_PBUF + 1;
 constexpr int SMEM_BYTES3 = STAGES3 * STAGE_BYTES3 + STAGING_BYTES + 1024 + 256;
 static_assert(SMEM_BYTES3 <= 232448, "exceeds the per-block shared-memory limit");
-static_assert(NUM_BARS3 * 8 + 12 <= 256, "barrier area");
+static_assert(NUM_BARS3 * 8 + 8 <= 256, "barrier area");
 static_assert(TMEM_COLS3 == 512, "TMEM allocation is a power of two");
 
 // fp32 D, TF32 A and B, A K-major, B K- or MN-major, M = 256, N = 128.
@@ -201,14 +201,13 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
   uint8_t* staging = smem + STAGES3 * STAGE_BYTES3;  // per epilogue warp: two 2 KB boxes
   uint64_t* bars = reinterpret_cast<uint64_t*>(staging + STAGING_BYTES);
   uint64_t* full_bar = bars;                                   // [STAGES3] this CTA's loads landed
-  uint64_t* conv_bar = bars + STAGES3;                         // [STAGES3] both CTAs split the stage (leader)
+  uint64_t* conv_bar = bars + STAGES3;                         // [STAGES3] all converter warps split the stage (leader)
   uint64_t* empty_bar = bars + 2 * STAGES3;                    // [STAGES3] MMAs done with the stage (both CTAs)
   uint64_t* pfull_bar = bars + 3 * STAGES3;                    // [NUM_PBUF] k-block sum ready (both CTAs)
   uint64_t* pempty_bar = bars + 3 * STAGES3 + NUM_PBUF;        // [NUM_PBUF] k-block sum folded (leader)
   uint64_t* drain_bar = bars + 3 * STAGES3 + 2 * NUM_PBUF;     // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* conv_ok = reinterpret_cast<volatile int*>(tmem_slot + 2);  // converters' shared wait result
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();  // 0 = leader, 1 = peer
@@ -218,7 +217,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES3; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
-      mbar_init(smem_u32(&conv_bar[s]), 2);
+      mbar_init(smem_u32(&conv_bar[s]), 2 * NUM_CONV_WARPS);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int a = 0; a < NUM_PBUF; ++a) {
@@ -369,29 +368,31 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- converters (both CTAs)
-    const int ct = threadIdx.x - 32 * (2 + NUM_EPI_WARPS);
+    // Each converter warp splits its own quarter of every stage and signals
+    // the leader itself, so the warps pipeline across stages: no named
+    // barrier, one arrival per warp and CTA on the leader's barrier.
+    const int cw = warp - (2 + NUM_EPI_WARPS);
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int t = pair; t < p.total_tiles && ok; t += npairs) {
       for (int kb = 0; kb < num_kb; ++kb) {
-        // one thread waits and the named barrier passes the result (and the
-        // landed data) on, so all converter threads leave the loop together
-        if (ct == 0) *conv_ok = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.timeout_ns) ? 1 : 0;
-        asm volatile("bar.sync 1, %0;" ::"n"(CONV_THREADS) : "memory");
-        if (!*conv_ok) { ok = false; break; }
+        // every lane waits itself (acquiring the landed bytes); the vote keeps
+        // the warp together if the wait runs out for some lanes only
+        const bool got = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.timeout_ns);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         float4* raw = reinterpret_cast<float4*>(smem + stage * STAGE_BYTES3);
         float4* lo = raw + RAW_BYTES / 16;
 #pragma unroll 4
-        for (int i = ct; i < RAW_BYTES / 16; i += CONV_THREADS) {
+        for (int i = cw * 32 + lane; i < RAW_BYTES / 16; i += CONV_THREADS) {
           const float4 x = raw[i];
           const float4 h = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
           raw[i] = h;
           lo[i] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
         }
-        fence_async_smem();  // the tensor core reads what these threads wrote
-        asm volatile("bar.sync 1, %0;" ::"n"(CONV_THREADS) : "memory");
-        if (ct == 0) remote_arrive(leader_conv + stage * 8);
+        fence_async_smem();  // the tensor core reads what these lanes wrote
+        __syncwarp();
+        if (lane == 0) remote_arrive(leader_conv + stage * 8);
         if (++stage == STAGES3) { stage = 0; phase ^= 1u; }
       }
     }
