@@ -45,7 +45,7 @@ METRIC = "NS-orthogonalization ms/optimizer-step & effective TFLOP/s (% of bf16 
 # traffic grows with the matrix count.  Reset an entry to None whenever its
 # kernel changes until a new capture is taken.
 PRODUCT_TRAFFIC_PER_LAUNCH = {("kimi-k2", "bf16"): 18.89e9,
-                              ("dense16", "fp32"): None, ("dense", "fp32"): None}
+                              ("dense16", "fp32"): 320.4e6, ("dense", "fp32"): 4 * 320.4e6}
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
