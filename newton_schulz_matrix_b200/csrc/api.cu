@@ -232,6 +232,8 @@ int chain_dtype(const muon_ns_params* ns) {
   return ns->mode == MUON_NS_STANDARD ? ns->compute_dtype : ns->gram_dtype;
 }
 
+double flops_of(int rows, int cols, const muon_ns_params* ns);  // algorithmic FLOPs of one matrix's chain
+
 // fp32 chains whose matrices fit in one CTA's shared memory run as a single
 // fused launch (one CTA per matrix); MUON_FUSED_SMALL=0 keeps the chained
 // products instead.
@@ -257,9 +259,7 @@ int run_fused_small(const Ctx& c, const Layout& L, const Bufs& B, int chunk, con
   a.restart_after = ns->mode == MUON_NS_GRAM_STABILIZED ? ns->restart_after : 0;
   a.iters = ns->iters;
   for (int i = 0; i < 3 * ns->iters; ++i) a.coeffs[i] = ns->coeffs[i];
-  const double n = L.n, m = L.m, K = ns->iters;
-  const double flops = a.mode == 0 ? K * (4.0 * m * n * n + 2.0 * n * n * n) : 0.0;
-  ProfScope ps(kProfFusedSmall, flops * chunk, 2.0 * chunk * n * m * 4, c.s);
+  ProfScope ps(kProfFusedSmall, flops_of(L.n, L.m, ns) * chunk, 2.0 * chunk * L.n * L.m * 4, c.s);
   return launch_fused_small(a, c.s);
 }
 
