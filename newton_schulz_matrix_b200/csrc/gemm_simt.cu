@@ -100,16 +100,15 @@ int gemm_simt(const GemmDesc& g, cudaStream_t s) {
   return (int)cudaGetLastError();
 }
 
-
-
-
 // ----------------------------------------------------------------------------
 // Fused fp32 chain for small matrices: one CTA per matrix runs every product of
 // the iteration in shared memory, so the whole Newton-Schulz chain is a single
 // launch.  The products are the same as the chained kernels' (standard form:
 // A = X X^T, B = b A + c A A, X <- a X + B X; Gram form: R = X X^T,
 // Q = a I + b R + c R R, Q_acc <- Q Q_acc, R <- (Q R) Q, restart, X = Q_acc X0),
-// here with plain R R (no symmetric shortcut is needed in shared memory).
+// here every product is formed in full (R R, not the R R^T of the chained
+// path, so R needs no exact symmetry).  The norm f = 1/(||U|| + eps) scales X0
+// as it is loaded.
 // ----------------------------------------------------------------------------
 namespace {
 
