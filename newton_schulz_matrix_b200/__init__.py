@@ -400,8 +400,11 @@ class StreamedMuonStep:
     """A Muon step fed from and returned to pinned host memory, with the PCIe
     copies overlapped with the orthogonalisation.
 
-    The parameters are cut into slices of consecutive tensors (at most
-    ``slice_bytes`` of gradients each).  Per slice, one stream copies the
+    The parameters are cut into slices (at most ``slice_bytes`` of gradients
+    each), taken in order of decreasing short side: the orthogonalisation's
+    work per byte grows with it, so the first slices give the next slices'
+    copies the most compute to hide behind, and the last slices, whose
+    copies cannot be hidden, are the cheapest.  Per slice, one stream copies the
     gradients host -> device, the compute stream runs the fused step on the
     slice, and a third stream copies the updated weights device -> host, so
     slice k's step runs while slice k+1's gradients arrive and slice k-1's
@@ -412,7 +415,7 @@ class StreamedMuonStep:
     waits for the whole step at the end of each call.
     """
 
-    def __init__(self, params, grads, moms, host_grads, host_params, *, slice_bytes: int = 2 << 30,
+    def __init__(self, params, grads, moms, host_grads, host_params, *, slice_bytes: int = 512 << 20,
                  workspace_bytes: int | None = None, **hp):
         if not (len(params) == len(grads) == len(moms) == len(host_grads) == len(host_params)):
             raise MuonError("params, grads, moms and their host copies must have equal lengths")
@@ -422,17 +425,21 @@ class StreamedMuonStep:
         dev = params[0].device
         self.params, self.grads = list(params), list(grads)
         self.host_grads, self.host_params = list(host_grads), list(host_params)
+        order = sorted(range(len(self.grads)), key=lambda i: (-min(self.grads[i].shape[-2:]), i))
         self.slices = []
-        start, acc = 0, 0
-        for i, g in enumerate(self.grads):
-            b = g.numel() * g.element_size()
-            if i > start and acc + b > slice_bytes:
-                self.slices.append((start, i))
-                start, acc = i, 0
+        cur, acc = [], 0
+        for i in order:
+            b = self.grads[i].numel() * self.grads[i].element_size()
+            if cur and acc + b > slice_bytes:
+                self.slices.append(cur)
+                cur, acc = [], 0
+            cur.append(i)
             acc += b
-        self.slices.append((start, len(self.grads)))
-        self.steps = [MuonStep(self.params[a:b], self.grads[a:b], list(moms[a:b]), workspace=None,
-                               workspace_bytes=1, **hp) for a, b in self.slices]
+        if cur:
+            self.slices.append(cur)
+        self.steps = [MuonStep([self.params[i] for i in idx], [self.grads[i] for i in idx],
+                               [moms[i] for i in idx], workspace=None, workspace_bytes=1, **hp)
+                      for idx in self.slices]
         need = max(st.workspace_needed[1] for st in self.steps)
         if workspace_bytes is not None:
             need = max(max(st.workspace_needed[0] for st in self.steps), min(need, int(workspace_bytes)))
@@ -451,11 +458,11 @@ class StreamedMuonStep:
         for s in (self.h2d, self.compute, self.d2h):
             s.wait_stream(caller)
         done = []
-        for k, (a, b) in enumerate(self.slices):
+        for k, idx in enumerate(self.slices):
             with torch.cuda.stream(self.h2d):
                 if self._computed[k] is not None:
                     self.h2d.wait_event(self._computed[k])
-                for i in range(a, b):
+                for i in idx:
                     self.grads[i].copy_(self.host_grads[i], non_blocking=True)
                 arrived = torch.cuda.Event()
                 arrived.record(self.h2d)
@@ -468,7 +475,7 @@ class StreamedMuonStep:
             self._computed[k] = ev
             with torch.cuda.stream(self.d2h):
                 self.d2h.wait_event(ev)
-                for i in range(a, b):
+                for i in idx:
                     self.host_params[i].copy_(self.params[i], non_blocking=True)
                 out = torch.cuda.Event()
                 out.record(self.d2h)
