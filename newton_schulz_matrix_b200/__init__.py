@@ -22,7 +22,7 @@ __all__ = [
     "MuonError", "load_library", "library_path", "muon_step", "muon_ns_batched",
     "muon_workspace_size", "muon_workspace_min", "muon_ns_workspace_size", "muon_ns_flops",
     "muon_status_string", "muon_profile_begin", "muon_profile_end", "MuonStep", "StreamedMuonStep",
-    "muon_ns_batched_noalloc",
+    "plan_slices", "muon_ns_batched_noalloc",
     "NOALLOC_SCRATCH_BYTES", "EXPORTED_SYMBOLS",
 ]
 
@@ -396,6 +396,24 @@ def muon_ns_batched_noalloc(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5,
     _raise(rc, "muon_ns_batched_noalloc")
 
 
+def plan_slices(shapes, nbytes, slice_bytes):
+    """Slices of the streamed step: lists of tensor indices, at most
+    ``slice_bytes`` each (a larger tensor gets a slice of its own), taken in
+    order of decreasing short side (ties by index), so that the slices with
+    the most orthogonalisation work per byte come first."""
+    order = sorted(range(len(shapes)), key=lambda i: (-min(shapes[i][-2:]), i))
+    slices, cur, acc = [], [], 0
+    for i in order:
+        if cur and acc + nbytes[i] > slice_bytes:
+            slices.append(cur)
+            cur, acc = [], 0
+        cur.append(i)
+        acc += nbytes[i]
+    if cur:
+        slices.append(cur)
+    return slices
+
+
 class StreamedMuonStep:
     """A Muon step fed from and returned to pinned host memory, with the PCIe
     copies overlapped with the orthogonalisation.
@@ -425,18 +443,8 @@ class StreamedMuonStep:
         dev = params[0].device
         self.params, self.grads = list(params), list(grads)
         self.host_grads, self.host_params = list(host_grads), list(host_params)
-        order = sorted(range(len(self.grads)), key=lambda i: (-min(self.grads[i].shape[-2:]), i))
-        self.slices = []
-        cur, acc = [], 0
-        for i in order:
-            b = self.grads[i].numel() * self.grads[i].element_size()
-            if cur and acc + b > slice_bytes:
-                self.slices.append(cur)
-                cur, acc = [], 0
-            cur.append(i)
-            acc += b
-        if cur:
-            self.slices.append(cur)
+        self.slices = plan_slices([tuple(g.shape) for g in self.grads],
+                                  [g.numel() * g.element_size() for g in self.grads], slice_bytes)
         self.steps = [MuonStep([self.params[i] for i in idx], [self.grads[i] for i in idx],
                                [moms[i] for i in idx], workspace=None, workspace_bytes=1, **hp)
                       for idx in self.slices]

@@ -50,3 +50,18 @@ def test_traffic_is_only_reported_for_captured_workloads():
 def test_weak_scaling_value_is_all_ranks_work_over_the_slowest_step():
     assert bench.whole_job_tflops(4, 513.2e12, 400.0) == pytest.approx(4 * 513.2e12 / 0.4 / 1e12)
     assert bench.max_over_ranks(12.5, None, None) == 12.5
+
+
+def test_streamed_slices_take_the_widest_short_side_first_and_respect_the_budget():
+    from newton_schulz_matrix_b200 import plan_slices
+    shapes = [(2048, 7168)] * 3 + [(7168, 2048)] + [(7168, 18432)] * 2 + [(64, 128)]
+    nbytes = [r * c * 2 for r, c in shapes]
+    slices = plan_slices(shapes, nbytes, 64 << 20)
+    flat = [i for sl in slices for i in sl]
+    assert sorted(flat) == list(range(len(shapes)))              # every tensor exactly once
+    assert flat[:2] == [4, 5]                                    # n = 7168 first
+    assert flat[-1] == 6                                         # the 64 x 128 matrix last
+    for sl in slices:                                            # budget, or a single oversized tensor
+        assert len(sl) == 1 or sum(nbytes[i] for i in sl) <= 64 << 20
+    assert [len(sl) for sl in slices] == [1, 1, 2, 3]             # 29 MB experts pair up (the small one joins); 264 MB dense alone
+    assert plan_slices([], [], 1) == []
