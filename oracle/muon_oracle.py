@@ -41,9 +41,10 @@ Readings where the pages are silent or garbled (each is listed in the design doc):
 
 Parity pins: every function below is pinned by ``tests/test_oracle_pins.py``
 against closed forms, an SVD routine, exact algebraic identities or values the
-pages print; see that file.  The Gram FLOP counters are the one exception:
-"parity unpinned" (the pages' complexity table was lost; only its 42-58 % band
-survives and is used as a plausibility check).
+pages print; see that file.  The Gram FLOP counters are pinned to the products
+the Gram iteration below executes (an instrumented run counts them), not to the
+pages: their complexity table was lost, and only its 42-58 % band survives, as a
+plausibility check.
 """
 from __future__ import annotations
 
@@ -275,8 +276,8 @@ def flops_standard(rows: int, cols: int, iters: int) -> int:
 
 
 def flops_gram(rows: int, cols: int, iters: int, restart_after: int = 0) -> int:
-    """Products the Gram iteration above executes (parity unpinned: the pages'
-    own complexity table was lost).
+    """Products the Gram iteration above executes (pinned to an instrumented
+    run of that iteration; the pages' own complexity table was lost).
 
     R0 = X0 X0^T (2mn^2); per k: R^2 (2n^3), Q Q_acc (2n^3, skipped at k = 1 and
     right after a restart, where Q_acc = I); R update Q R Q (4n^3) for k < K

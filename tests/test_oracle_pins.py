@@ -70,8 +70,9 @@ def test_kimi_k2_total_flops():
 
 
 def test_gram_flops_plausibility_band():
-    """Parity unpinned: the pages' complexity table was lost.  Our counts must
-    give savings that include the surviving 42-58 % band somewhere in alpha > 1."""
+    """The pages' complexity table was lost (our counts are pinned to the
+    executed products below).  They must give savings that include the
+    surviving 42-58 % band somewhere in alpha > 1."""
     band = FACTS["gram_flop_saving_band"]
     n = 1024
     savings = []
@@ -329,3 +330,88 @@ def test_fp16_gram_negative_eigenvalues_and_restart():
     assert abs(naive[-1]) > 10 * abs(stab[-1])
     ref = oracle.ns_standard(X0, Q5_)
     assert rel(outs[0], ref) > 3 * rel(outs[2], ref)
+
+
+# ---------------------------------------------------------------------------
+# FLOP counters pinned to the products the iteration actually executes: the
+# oracle's own iteration runs on an array wrapper that counts every matrix
+# product (2 * rows * cols * inner), skipping products with an exact identity
+# operand (Q_acc = I at k = 1 and right after a restart, which the kernels skip)
+# ---------------------------------------------------------------------------
+class _Counted:
+    __array_ufunc__ = None  # numpy's operators defer to the reflected methods below
+    flops = [0]
+
+    def __init__(self, a):
+        self.a = np.asarray(a, dtype=np.float64)
+
+    @staticmethod
+    def _raw(x):
+        return x.a if isinstance(x, _Counted) else np.asarray(x)
+
+    @classmethod
+    def _count(cls, A, B):
+        eye = lambda M: M.ndim == 2 and M.shape[0] == M.shape[1] and np.array_equal(M, np.eye(M.shape[0]))
+        if not (eye(A) or eye(B)):
+            cls.flops[0] += 2 * A.shape[0] * B.shape[1] * A.shape[1]
+        return _Counted(A @ B)
+
+    def __matmul__(self, o):
+        return self._count(self.a, self._raw(o))
+
+    def __rmatmul__(self, o):
+        return self._count(self._raw(o), self.a)
+
+    def __add__(self, o):
+        return _Counted(self.a + self._raw(o))
+
+    __radd__ = __add__
+
+    def __sub__(self, o):
+        return _Counted(self.a - self._raw(o))
+
+    def __rsub__(self, o):
+        return _Counted(self._raw(o) - self.a)
+
+    def __mul__(self, o):
+        return _Counted(self.a * self._raw(o))
+
+    __rmul__ = __mul__
+
+    @property
+    def T(self):
+        return _Counted(self.a.T)
+
+    @property
+    def shape(self):
+        return self.a.shape
+
+    def copy(self):
+        return _Counted(self.a.copy())
+
+
+@pytest.mark.parametrize("shape", [(8, 24), (24, 8), (16, 16), (12, 40)])
+@pytest.mark.parametrize("iters,restart", [(5, 0), (5, 2), (3, 1), (6, 4), (1, 0), (2, 0)])
+def test_gram_flop_count_equals_the_products_executed(monkeypatch, shape, iters, restart):
+    from oracle import muon_oracle as mo
+    monkeypatch.setattr(mo, "_f64", lambda a: _Counted(a))
+    X0 = np.random.default_rng(3).standard_normal(shape)
+    X0 = X0 if shape[0] <= shape[1] else X0.T  # the iteration runs on the n x m orientation
+    X0 = X0 / np.linalg.norm(X0)
+    _Counted.flops[0] = 0
+    out = mo.ns_gram(X0, [oracle.QUINTIC] * iters, restart_after=restart)
+    assert isinstance(out, _Counted)
+    assert _Counted.flops[0] == oracle.flops_gram(*shape, iters, restart)
+    mode = oracle.GRAM if restart == 0 else oracle.GRAM_STABILIZED
+    if restart == 0 or restart < iters:
+        assert _Counted.flops[0] == oracle.flops(*shape, iters, mode, restart_after=restart or 2)
+
+
+@pytest.mark.parametrize("shape", [(8, 24), (16, 16)])
+def test_standard_flop_count_equals_the_products_executed(monkeypatch, shape):
+    from oracle import muon_oracle as mo
+    monkeypatch.setattr(mo, "_f64", lambda a: _Counted(a))
+    _Counted.flops[0] = 0
+    X0 = np.random.default_rng(4).standard_normal(shape)
+    mo.ns_standard(X0 / np.linalg.norm(X0), [oracle.QUINTIC] * 5)
+    assert _Counted.flops[0] == oracle.flops_standard(*shape, 5)
