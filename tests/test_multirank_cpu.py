@@ -63,6 +63,32 @@ def _sharded_worker(rank, world, port, q):
     dist.destroy_process_group()
 
 
+def _idle_rank_worker(rank, world, port, q):
+    """Three ranks, two matrices: one rank owns nothing and only receives."""
+    _init(rank, world, port)
+    torch.manual_seed(1)
+    shapes = [(32, 64), (48, 48)]
+    params = [torch.randn(*s) for s in shapes]
+    grads = [torch.randn(*s) for s in shapes]
+    start = [p.clone() for p in params]
+    owner = lpt_owners([ns_cost(s) for s in shapes], world)
+    moms = {i: torch.zeros(*shapes[i]) for i in range(len(shapes)) if owner[i] == rank}
+
+    def fake_local(ps, gs, ms, **hp):
+        def run():
+            for p, g in zip(ps, gs):
+                p.sub_(g)
+        return run
+
+    step = ShardedMuonStep(params, grads, moms, local_step_factory=fake_local)
+    step()
+    step()  # a second step: the idle rank keeps taking the same collective steps
+    ok = all(torch.equal(params[i], (start[i] - grads[i]) - grads[i]) for i in range(len(shapes)))
+    q.put((rank, ok, step.owned()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def _spawn(fn, world=2):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -103,3 +129,11 @@ def test_lpt_balances_the_kimi_k2_set():
     assert lpt_owners([5, 5, 5], 1) == [0, 0, 0]
     with pytest.raises(ValueError):
         lpt_owners([1.0], 0)
+
+
+def test_sharded_step_with_a_rank_that_owns_nothing():
+    out = _spawn(_idle_rank_worker, world=3)
+    assert [ok for _, ok, _ in out] == [True, True, True]
+    owned = [o for _, _, o in out]
+    assert sorted(i for o in owned for i in o) == [0, 1]
+    assert [] in owned
