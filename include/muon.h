@@ -14,10 +14,13 @@
  * Conventions shared by every entry point
  *   - Every matrix is dense row-major in device memory (leading dimension =
  *     cols) and 16-byte aligned.  The caller owns all memory, including the
- *     workspace; the library allocates nothing and keeps no state between
- *     calls.
+ *     workspace; the library allocates nothing and carries no data from one
+ *     call to the next (it only caches per-device launch settings on first
+ *     use: the SM count, shared-memory opt-ins, how many CTA pairs fit).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *     default stream) and take no locks.  The return value reports argument
+ *     default stream).  They take no lock on the launch path; the opt-in
+ *     profiler and the allocation-free entry point's one-time scratch lookup
+ *     take a mutex.  The return value reports argument
  *     and launch errors only (MUON_OK, MUON_ERR_*).  Conditions found on the
  *     device are OR-ed into the optional per-matrix status words (device int
  *     array, one per matrix, zeroed by the call): MUON_STATUS_NONFINITE when

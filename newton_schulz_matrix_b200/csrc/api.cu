@@ -3,7 +3,12 @@
 // the workspace layout, and the launch sequence of one Muon step:
 //
 //   pack (momentum, Nesterov, orientation, sums of squares)  -> norm
-//   -> Newton-Schulz chain of tensor-core products            -> unpack (update)
+//   -> Newton-Schulz chain                                    -> unpack (update)
+//
+// The chain's products run on the tensor cores: tcgen05 kind::f16 for bf16 and
+// fp16 storage, 3xTF32 (kind::tf32) for fp32 storage with n >= 256.  An fp32
+// chain of matrices small enough for one CTA's shared memory runs as a single
+// fused launch, and the remaining fp32 products run on a CUDA-core kernel.
 //
 // The iteration order follows the "Gram Newton-Schulz" write-up (standard
 // form: A = X X^T, B = b A + c A^2, X = a X + B X; Gram form: iterate on
