@@ -270,7 +270,15 @@ def muon_ns_workspace_size(count: int, rows: int, cols: int, coeffs=(QUINTIC,) *
 def muon_ns_batched(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2,
                     eps=1e-7, compute_dtype=None, gram_dtype="fp16", workspace: torch.Tensor | None = None,
                     status: torch.Tensor | None = None, stream=None) -> None:
-    """Orthogonalise same-shape matrices in place (result has each input's shape)."""
+    """Orthogonalise same-shape matrices in place (result has each input's shape).
+
+    ``compute_dtype`` is the storage type of the chain: None picks "fp32" for
+    fp32 inputs and "bf16" otherwise; "fp16" is also accepted.  fp32 chains run
+    3xTF32 tensor-core products when the short side is at least 256, and a
+    single fused launch per call for matrices small enough for one block's
+    shared memory.  ``gram_dtype`` is the 16-bit type of the Gram chains.
+    ``status``, if given, is an int32 CUDA tensor with one word per matrix.
+    """
     lib = load_library()
     if len(X) == 0:
         return
