@@ -27,7 +27,7 @@ Sources (web pages, cited by title and section):
   paragraph (float16 Gram iteration, restart after step 2, re-initialise the
   Gram matrix).
 
-Readings where the pages are silent or garbled (each is listed in the design doc):
+Readings where the pages are silent or garbled:
 
 * Normalisation is X0 = U / (||U||_F + eps) without the listing's extra sqrt(m)
   factor (the listing's cubic form needs it, the quintic coefficients do not).
@@ -36,7 +36,10 @@ Readings where the pages are silent or garbled (each is listed in the design doc):
   X_k = Q_k X_{k-1}, R_k = Q_k R_{k-1} Q_k and X_K = (Q_K ... Q_1) X_0.
 * The accumulated product is formed by left multiplication Q_acc <- Q_k Q_acc.
 * "Restart after step 2" is one restart after iteration ``restart_after``
-  (default 2): X <- Q_acc X0, R <- X X^T, Q_acc <- I, then continue.
+  (default 2): X <- Q_acc X0, R <- X X^T, Q_acc <- I, then continue.  The
+  periodic reading ("re-initialise the Gram matrix" every few steps) is the
+  option ``restart_every`` = e > 0: restarts after iterations restart_after,
+  restart_after + e, restart_after + 2e, ... while they are before the last.
 * Nesterov (not on the pages) is U = (1 - mu) G + mu M_new.
 
 Parity pins: every function below is pinned by ``tests/test_oracle_pins.py``
@@ -69,15 +72,14 @@ def _f64(a) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Optional storage-rounding emulation (diagnosis only, never used for grading)
+# Storage rounding (used by the stored-precision iteration further down)
 # ---------------------------------------------------------------------------
 def round_to(x: np.ndarray, fmt: str | None) -> np.ndarray:
     """Round ``x`` to a storage format and back to float64.
 
     ``fmt`` is None (no rounding), "fp32", "bf16" (round-to-nearest-even on the
     float32 bit pattern, top 16 bits kept) or "fp16" (IEEE binary16, overflow to
-    inf).  Used only to *diagnose* where a reduced-precision GPU result departs
-    from the exact iteration; parity is always graded against fmt=None.
+    inf).
     """
     if fmt is None:
         return x
@@ -144,26 +146,34 @@ def frobenius_normalize(X: np.ndarray, eps: float = 1e-7) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Step a5: standard odd-polynomial Newton-Schulz   [GramNS, standard iteration]
 # ---------------------------------------------------------------------------
-def ns_standard(X0: np.ndarray, coeffs: Sequence[Sequence[float]], emulate: str | None = None) -> np.ndarray:
+def ns_standard(X0: np.ndarray, coeffs: Sequence[Sequence[float]]) -> np.ndarray:
     """Iterate X <- a X + (b A + c A A) X with A = X X^T, once per (a, b, c)."""
     X = _f64(X0)
     for a, b, c in coeffs:
-        A = round_to(X @ X.T, emulate)                 # n x n, 2 m n^2 flops
-        B = round_to(b * A + c * (A @ A), emulate)      # n x n, 2 n^3 flops
-        X = round_to(a * X + B @ X, emulate)            # n x m, 2 m n^2 flops
+        A = X @ X.T                 # n x n, 2 m n^2 flops
+        B = b * A + c * (A @ A)     # n x n, 2 n^3 flops
+        X = a * X + B @ X           # n x m, 2 m n^2 flops
     return X
 
 
 # ---------------------------------------------------------------------------
 # Steps a6/a7: Gram Newton-Schulz, naive and stabilised   [GramNS, Gram rewrite]
 # ---------------------------------------------------------------------------
+def is_restart(k: int, iters: int, restart_after: int, restart_every: int = 0) -> bool:
+    """Whether the stabilised Gram iteration restarts after iteration k (1-based)."""
+    if not restart_after or k >= iters or k < restart_after:
+        return False
+    if k == restart_after:
+        return True
+    return restart_every > 0 and (k - restart_after) % restart_every == 0
+
+
 def ns_gram(
     X0: np.ndarray,
     coeffs: Sequence[Sequence[float]],
     restart_after: int = 0,
-    emulate_gram: str | None = None,
-    emulate_x: str | None = None,
     trace: list | None = None,
+    restart_every: int = 0,
 ) -> np.ndarray:
     """Gram form of the same iteration.
 
@@ -171,31 +181,31 @@ def ns_gram(
     if k == restart_after (and k < K): X0 <- Q_acc X0, R <- X0 X0^T, Q_acc <- I;
     elif k < K: R <- Q R Q.  Finally X = Q_acc X0.
 
-    ``restart_after = 0`` is the naive variant, 2 the stabilised one.
-    ``emulate_gram`` / ``emulate_x`` round the stored n x n and n x m matrices
-    (diagnosis only).  If ``trace`` is a list, (k, R, Q_acc, X0) is appended after
-    each iteration k, with R the Gram matrix the next iteration will use.
+    ``restart_after = 0`` is the naive variant, 2 the stabilised one;
+    ``restart_every`` > 0 repeats the restart (see ``is_restart``).
+    If ``trace`` is a list, (k, R, Q_acc, X0) is appended after each iteration
+    k, with R the Gram matrix the next iteration will use.
     """
     X = _f64(X0)
     n = X.shape[0]
     eye = np.eye(n)
-    R = round_to(X @ X.T, emulate_gram)
+    R = X @ X.T
     Qacc = eye.copy()
     K = len(coeffs)
     for k, (a, b, c) in enumerate(coeffs, start=1):
-        Q = round_to(a * eye + b * R + c * (R @ R), emulate_gram)
-        Qacc = round_to(Q @ Qacc, emulate_gram)
+        Q = a * eye + b * R + c * (R @ R)
+        Qacc = Q @ Qacc
         if k == K:
             break
-        if restart_after and k == restart_after:
-            X = round_to(Qacc @ X, emulate_x)
-            R = round_to(X @ X.T, emulate_gram)
+        if is_restart(k, K, restart_after, restart_every):
+            X = Qacc @ X
+            R = X @ X.T
             Qacc = eye.copy()
         else:
-            R = round_to(round_to(Q @ R, emulate_gram) @ Q, emulate_gram)
+            R = (Q @ R) @ Q
         if trace is not None:
             trace.append((k, R.copy(), Qacc.copy(), X.copy()))
-    return round_to(Qacc @ X, emulate_x)
+    return Qacc @ X
 
 
 # ---------------------------------------------------------------------------
@@ -207,6 +217,7 @@ def newton_schulz(
     mode: str = STANDARD,
     restart_after: int = 2,
     eps: float = 1e-7,
+    restart_every: int = 0,
 ) -> np.ndarray:
     """Orthogonalise one 2-D matrix; the result has U's storage shape."""
     if mode not in MODES:
@@ -221,8 +232,86 @@ def newton_schulz(
     elif mode == GRAM:
         X = ns_gram(X0, coeffs, restart_after=0)
     else:
-        X = ns_gram(X0, coeffs, restart_after=restart_after)
+        X = ns_gram(X0, coeffs, restart_after=restart_after, restart_every=restart_every)
     return unorient(X, transposed)
+
+
+# ---------------------------------------------------------------------------
+# The same iterations with 16-bit storage between the products
+# ---------------------------------------------------------------------------
+# The pages fix no storage precision beyond "float16" for the stabilised Gram
+# variant [GramNS].  A 16-bit execution computes every product exactly enough
+# (fp32 accumulation) and rounds it once, to nearest-even, when it stores it.
+# The two functions below state that execution in fp64 with the rounding at
+# those store points, so that the error such an execution cannot avoid on a
+# given input (its floor) can be measured.  They are not the oracle the GPU
+# results are graded against: ``ns_standard`` / ``ns_gram`` are.
+#
+# Store points, per product (f = prescale applies only while X is the raw U):
+#   standard:  A = f^2 X X^T (symmetric);  B = c A A^T + b A (symmetric, only
+#              if c != 0);  X = f (a X + B X), or f (a X + b (A X)) if c == 0
+#   Gram:      R = f^2 X X^T (symmetric);  Q = c R R^T + b R + a I (symmetric);
+#              Q_acc = Q (first after a start) or Q Q_acc;  T = Q R;
+#              R = T Q (symmetric);  restart: X = f Q_acc X, R = X X^T;
+#              result f Q_acc X
+# A symmetric product is stored as its upper triangle mirrored onto the lower
+# one (the GPU computes only that triangle).  ``fmt`` "fp64" keeps every
+# product unrounded but otherwise runs the same steps.
+def _stored(x: np.ndarray, fmt: str, symmetric: bool = False) -> np.ndarray:
+    if symmetric:
+        x = np.triu(x) + np.triu(x, 1).T
+    return x if fmt == "fp64" else round_to(x, fmt)
+
+
+def ns_standard_stored(X: np.ndarray, coeffs: Sequence[Sequence[float]], fmt: str,
+                       prescale: float | None = None) -> np.ndarray:
+    """Standard iteration with every product stored in ``fmt``.
+
+    ``X`` is the stored input: either X0 already normalised (``prescale``
+    None) or the raw oriented U, in which case the first iteration applies
+    f = ``prescale`` = 1 / (||U||_F + eps) inside its stores.
+    """
+    X = _f64(X)
+    f = 1.0 if prescale is None else float(prescale)
+    for a, b, c in coeffs:
+        A = _stored(f * f * (X @ X.T), fmt, symmetric=True)
+        if c != 0.0:
+            B = _stored(c * (A @ A.T) + b * A, fmt, symmetric=True)
+            X = _stored(f * (a * X + B @ X), fmt)
+        else:
+            X = _stored(f * (a * X + b * (A @ X)), fmt)
+        f = 1.0
+    return X
+
+
+def ns_gram_stored(X: np.ndarray, coeffs: Sequence[Sequence[float]], fmt: str, restart_after: int = 0,
+                   prescale: float | None = None, trace: list | None = None, restart_every: int = 0) -> np.ndarray:
+    """Gram iteration (naive: ``restart_after`` 0) with every product stored in
+    ``fmt``; ``X`` and ``prescale`` as in ``ns_standard_stored``.  ``trace`` gets
+    (k, R, Q_acc, X) after each iteration k < K, as in ``ns_gram``."""
+    X = _f64(X)
+    n = X.shape[0]
+    eye = np.eye(n)
+    f = 1.0 if prescale is None else float(prescale)
+    R = _stored(f * f * (X @ X.T), fmt, symmetric=True)
+    Qacc = None  # identity
+    K = len(coeffs)
+    for k, (a, b, c) in enumerate(coeffs, start=1):
+        Q = _stored(c * (R @ R.T) + b * R + a * eye, fmt, symmetric=True)
+        Qacc = Q if Qacc is None else _stored(Q @ Qacc, fmt)
+        if k == K:
+            break
+        if is_restart(k, K, restart_after, restart_every):
+            X = _stored(f * (Qacc @ X), fmt)
+            f = 1.0
+            R = _stored(X @ X.T, fmt, symmetric=True)
+            Qacc = None
+        else:
+            T = _stored(Q @ R, fmt)
+            R = _stored(T @ Q, fmt, symmetric=True)
+        if trace is not None:
+            trace.append((k, R.copy(), eye.copy() if Qacc is None else Qacc.copy(), X.copy()))
+    return _stored(f * (Qacc @ X), fmt)
 
 
 # ---------------------------------------------------------------------------
@@ -252,11 +341,12 @@ def muon_step(
     coeffs: Sequence[Sequence[float]],
     mode: str = STANDARD,
     restart_after: int = 2,
+    restart_every: int = 0,
 ) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
     """One Muon step for one parameter: returns (W_new, M_new, O)."""
     M_new = momentum_update(M, G, momentum)
     U = nesterov_blend(G, M_new, momentum, nesterov)
-    O = newton_schulz(U, coeffs, mode=mode, restart_after=restart_after, eps=eps)
+    O = newton_schulz(U, coeffs, mode=mode, restart_after=restart_after, eps=eps, restart_every=restart_every)
     r, c = np.shape(W)
     W_new = apply_update(W, O, lr, weight_decay, update_scale(r, c, scale_coef))
     return W_new, M_new, O
@@ -275,13 +365,13 @@ def flops_standard(rows: int, cols: int, iters: int) -> int:
     return iters * flops_standard_iteration(rows, cols)
 
 
-def flops_gram(rows: int, cols: int, iters: int, restart_after: int = 0) -> int:
+def flops_gram(rows: int, cols: int, iters: int, restart_after: int = 0, restart_every: int = 0) -> int:
     """Products the Gram iteration above executes (pinned to an instrumented
     run of that iteration; the pages' own complexity table was lost).
 
     R0 = X0 X0^T (2mn^2); per k: R^2 (2n^3), Q Q_acc (2n^3, skipped at k = 1 and
     right after a restart, where Q_acc = I); R update Q R Q (4n^3) for k < K
-    unless k is the restart step, which instead costs Q_acc X0 (2mn^2) and
+    unless k is a restart step, which instead costs Q_acc X0 (2mn^2) and
     X X^T (2mn^2); finally Q_acc X0 (2mn^2).
     """
     n, m = min(rows, cols), max(rows, cols)
@@ -295,7 +385,7 @@ def flops_gram(rows: int, cols: int, iters: int, restart_after: int = 0) -> int:
         fresh = False
         if k == iters:
             break
-        if restart_after and k == restart_after:
+        if is_restart(k, iters, restart_after, restart_every):
             total += 2 * sq
             fresh = True
         else:
@@ -303,12 +393,12 @@ def flops_gram(rows: int, cols: int, iters: int, restart_after: int = 0) -> int:
     return total + sq
 
 
-def flops(rows: int, cols: int, iters: int, mode: str, restart_after: int = 2) -> int:
+def flops(rows: int, cols: int, iters: int, mode: str, restart_after: int = 2, restart_every: int = 0) -> int:
     if mode == STANDARD:
         return flops_standard(rows, cols, iters)
     if mode == GRAM:
         return flops_gram(rows, cols, iters, 0)
-    return flops_gram(rows, cols, iters, restart_after)
+    return flops_gram(rows, cols, iters, restart_after, restart_every)
 
 
 def singular_value_map(sigma: Iterable[float], coeffs: Sequence[Sequence[float]]) -> np.ndarray:

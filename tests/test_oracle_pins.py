@@ -140,6 +140,8 @@ def test_gram_equals_standard_in_exact_arithmetic(shape):
     assert rel(oracle.ns_gram(X0, Q5, 0), std) < 1e-12
     for r in (1, 2, 3, 4):
         assert rel(oracle.ns_gram(X0, Q5, r), std) < 1e-12
+        for e in (1, 2, 3):  # periodic restarts
+            assert rel(oracle.ns_gram(X0, Q5, r, restart_every=e), std) < 1e-12
     for K in range(1, 6):
         assert rel(oracle.ns_gram(X0, Q5[:K], 0), oracle.ns_standard(X0, Q5[:K])) < 1e-12
 
@@ -314,7 +316,7 @@ def test_fp16_gram_negative_eigenvalues_and_restart():
     """The write-up's stabilised-variant paragraph: in float16 the Gram matrix
     picks up negative eigenvalues that the naive iteration amplifies; restarting
     after step 2 (fresh R = X X^T) keeps them small.  Reproduced with the
-    oracle's fp16 storage emulation on an ill-conditioned input."""
+    oracle's fp16 stored-precision iteration on an ill-conditioned input."""
     Q5_ = [oracle.QUINTIC] * 5
     U = synth.with_spectrum(64, 256, synth.log_uniform_sigma(64, 1e-6, 1, 5), 9).double().numpy()
     X0 = oracle.frobenius_normalize(U)
@@ -322,14 +324,142 @@ def test_fp16_gram_negative_eigenvalues_and_restart():
     outs = {}
     for ra in (0, 2):
         tr = []
-        outs[ra] = oracle.ns_gram(X0, Q5_, ra, emulate_gram="fp16", emulate_x="bf16", trace=tr)
-        mins[ra] = [np.linalg.eigvalsh((R + R.T) / 2).min() for _, R, _, _ in tr]
+        outs[ra] = oracle.ns_gram_stored(oracle.round_to(X0, "fp16"), Q5_, "fp16", ra, trace=tr)
+        mins[ra] = [np.linalg.eigvalsh(R).min() for _, R, _, _ in tr]
     naive, stab = mins[0], mins[2]
     assert all(v < 0 for v in naive)
     assert all(abs(b / a) > 8 for a, b in zip(naive, naive[1:]))   # ~a^2 growth per step
     assert abs(naive[-1]) > 10 * abs(stab[-1])
     ref = oracle.ns_standard(X0, Q5_)
     assert rel(outs[0], ref) > 3 * rel(outs[2], ref)
+
+
+# ---------------------------------------------------------------------------
+# The stored-precision iterations (they set the bar of a few GPU tests on
+# ill-conditioned inputs), pinned two ways:
+#   - with no rounding ("fp64") they are the exact iteration, which the pins
+#     above tie to the SVD: this fixes their algebra, the mirrored triangles,
+#     and where f = 1 / (||U|| + eps) enters when they start from the raw U;
+#   - on diagonal inputs every product is a single multiplication per entry,
+#     so the iteration reduces to scalar recurrences with one rounding per
+#     stored product; written out below entry by entry, they must agree bit for
+#     bit.  A rounding too many or too few, or at the wrong point, changes the
+#     result (checked with planted variants).
+# ---------------------------------------------------------------------------
+SCHEDULES = {"quintic": Q5, "cubic": [oracle.CUBIC] * 4,
+             "mixed": [(3.0, -3.2, 1.2), oracle.CUBIC, oracle.QUINTIC, (2.5, -2.0, 0.6)]}
+
+
+@pytest.mark.parametrize("sched", sorted(SCHEDULES))
+@pytest.mark.parametrize("mode,ra,every", [("standard", 0, 0), ("gram", 0, 0), ("gram_stabilized", 1, 0),
+                                           ("gram_stabilized", 2, 0), ("gram_stabilized", 1, 2)])
+@pytest.mark.parametrize("raw", [False, True])
+def test_stored_iteration_without_rounding_is_the_exact_iteration(sched, mode, ra, every, raw):
+    coeffs = SCHEDULES[sched]
+    U = rng_matrix(24, 72, 41) * 37.0
+    f = 1.0 / (oracle.frobenius_norm(U) + 1e-7)
+    exact = oracle.newton_schulz(U, coeffs, mode=mode, restart_after=ra or 2, restart_every=every)
+    start, pre = (U, f) if raw else (U * f, None)
+    if mode == "standard":
+        got = oracle.ns_standard_stored(start, coeffs, "fp64", prescale=pre)
+    else:
+        got = oracle.ns_gram_stored(start, coeffs, "fp64", ra, prescale=pre, restart_every=every)
+    assert rel(got, exact) < 1e-12
+
+
+def _scalar_standard(d, coeffs, fmt, f, round_a=True):
+    rnd = lambda v: oracle.round_to(np.asarray(v, dtype=np.float64), fmt)
+    s = d.copy()
+    for a, b, c in coeffs:
+        A = f * f * (s * s)
+        A = rnd(A) if round_a else A
+        if c != 0.0:
+            B = rnd(c * (A * A) + b * A)
+            s = rnd(f * (a * s + B * s))
+        else:
+            s = rnd(f * (a * s + b * (A * s)))
+        f = 1.0
+    return s
+
+
+def _scalar_gram(d, coeffs, fmt, ra, f, round_t=True):
+    rnd = lambda v: oracle.round_to(np.asarray(v, dtype=np.float64), fmt)
+    s = d.copy()
+    r = rnd(f * f * (s * s))
+    qacc = None
+    for k, (a, b, c) in enumerate(coeffs, start=1):
+        q = rnd(c * (r * r) + b * r + a)
+        qacc = q if qacc is None else rnd(q * qacc)
+        if k == len(coeffs):
+            break
+        if ra and k == ra:
+            s = rnd(f * (qacc * s))
+            f = 1.0
+            r = rnd(s * s)
+            qacc = None
+        else:
+            t = q * r
+            t = rnd(t) if round_t else t
+            r = rnd(t * q)
+    return rnd(f * (qacc * s))
+
+
+def _diagonal_case(fmt, raw, n=400, m=560, seed=6):
+    """A diagonal n x m input whose scaled entries spread over [1e-4, 1] (entries
+    near 1 make every rounding visible); ``raw``: the stored values are 37.37 x
+    larger and the prescale brings them back (the store-point structure is what
+    is pinned here; the Frobenius normalisation is pinned by the fp64 test)."""
+    rng = np.random.default_rng(seed)
+    d = np.exp(rng.uniform(math.log(1e-4), 0.0, n)) * rng.choice([-1.0, 1.0], n)
+    scale = 37.37 if raw else 1.0
+    d = oracle.round_to(d * scale, fmt)
+    X = np.zeros((n, m))
+    X[np.arange(n), np.arange(n)] = d
+    f = 1.0 / float(np.max(np.abs(d))) if raw else None
+    return X, d, f
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp16"])
+@pytest.mark.parametrize("sched", sorted(SCHEDULES))
+@pytest.mark.parametrize("raw", [False, True])
+def test_stored_standard_rounds_exactly_at_the_store_points(fmt, sched, raw):
+    coeffs = SCHEDULES[sched]
+    X, d, f = _diagonal_case(fmt, raw)
+    got = oracle.ns_standard_stored(X, coeffs, fmt, prescale=f)
+    want = _scalar_standard(d, coeffs, fmt, 1.0 if f is None else f)
+    n = len(d)
+    assert np.array_equal(np.diag(got[:, :n]), want)
+    assert not np.any(got[:, :n] - np.diag(np.diag(got[:, :n]))) and not np.any(got[:, n:])
+    # planted variants: A kept unrounded, or f applied before the first store
+    assert not np.array_equal(_scalar_standard(d, coeffs, fmt, 1.0 if f is None else f, round_a=False), want)
+    if raw:
+        pre = oracle.round_to(d * f, fmt)
+        assert not np.array_equal(_scalar_standard(pre, coeffs, fmt, 1.0), want)
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "fp16"])
+@pytest.mark.parametrize("sched", ["quintic", "mixed"])
+@pytest.mark.parametrize("ra", [0, 1, 2])
+@pytest.mark.parametrize("raw", [False, True])
+def test_stored_gram_rounds_exactly_at_the_store_points(fmt, sched, ra, raw):
+    coeffs = SCHEDULES[sched]
+    X, d, f = _diagonal_case(fmt, raw, seed=7 + ra)
+    got = oracle.ns_gram_stored(X, coeffs, fmt, ra, prescale=f)
+    want = _scalar_gram(d, coeffs, fmt, ra, 1.0 if f is None else f)
+    n = len(d)
+    assert np.array_equal(np.diag(got[:, :n]), want)
+    assert not np.any(got[:, :n] - np.diag(np.diag(got[:, :n]))) and not np.any(got[:, n:])
+    assert not np.array_equal(_scalar_gram(d, coeffs, fmt, ra, 1.0 if f is None else f, round_t=False), want)
+
+
+def test_stored_symmetric_products_are_exactly_symmetric():
+    """The GPU stores X X^T, A A^T, R R^T and the R update's second product as
+    a mirrored upper triangle; the stored iteration's R must be too."""
+    U = synth.with_spectrum(32, 96, synth.log_uniform_sigma(32, 1e-4, 1, 3), 4).double().numpy()
+    tr = []
+    oracle.ns_gram_stored(oracle.round_to(oracle.frobenius_normalize(U), "fp16"), Q5, "fp16", 0, trace=tr)
+    for _, R, _, _ in tr:
+        assert np.array_equal(R, R.T)
 
 
 # ---------------------------------------------------------------------------
@@ -391,20 +521,38 @@ class _Counted:
 
 
 @pytest.mark.parametrize("shape", [(8, 24), (24, 8), (16, 16), (12, 40)])
-@pytest.mark.parametrize("iters,restart", [(5, 0), (5, 2), (3, 1), (6, 4), (1, 0), (2, 0)])
-def test_gram_flop_count_equals_the_products_executed(monkeypatch, shape, iters, restart):
+@pytest.mark.parametrize("iters,restart,every", [(5, 0, 0), (5, 2, 0), (3, 1, 0), (6, 4, 0), (1, 0, 0), (2, 0, 0),
+                                                 (5, 2, 2), (7, 1, 3), (5, 2, 1)])
+def test_gram_flop_count_equals_the_products_executed(monkeypatch, shape, iters, restart, every):
     from oracle import muon_oracle as mo
     monkeypatch.setattr(mo, "_f64", lambda a: _Counted(a))
     X0 = np.random.default_rng(3).standard_normal(shape)
     X0 = X0 if shape[0] <= shape[1] else X0.T  # the iteration runs on the n x m orientation
     X0 = X0 / np.linalg.norm(X0)
     _Counted.flops[0] = 0
-    out = mo.ns_gram(X0, [oracle.QUINTIC] * iters, restart_after=restart)
+    out = mo.ns_gram(X0, [oracle.QUINTIC] * iters, restart_after=restart, restart_every=every)
     assert isinstance(out, _Counted)
-    assert _Counted.flops[0] == oracle.flops_gram(*shape, iters, restart)
+    assert _Counted.flops[0] == oracle.flops_gram(*shape, iters, restart, every)
     mode = oracle.GRAM if restart == 0 else oracle.GRAM_STABILIZED
     if restart == 0 or restart < iters:
-        assert _Counted.flops[0] == oracle.flops(*shape, iters, mode, restart_after=restart or 2)
+        assert _Counted.flops[0] == oracle.flops(*shape, iters, mode, restart_after=restart or 2, restart_every=every)
+
+
+@pytest.mark.parametrize("iters,restart,every,points", [(5, 2, 2, [2, 4]), (7, 1, 3, [1, 4]), (5, 2, 1, [2, 3, 4]),
+                                                        (5, 2, 0, [2]), (5, 4, 1, [4]), (3, 2, 5, [2])])
+def test_periodic_restart_points(iters, restart, every, points):
+    """Restarts come after iteration restart_after and every restart_every
+    iterations after it, never after the last iteration; each restart leaves
+    Q_acc = I and R = X X^T of the materialised X (seen in the trace)."""
+    assert [k for k in range(1, iters + 1) if oracle.is_restart(k, iters, restart, every)] == points
+    X0 = oracle.frobenius_normalize(rng_matrix(12, 36, 8))
+    tr = []
+    out = oracle.ns_gram(X0, Q5[:1] * iters, restart, trace=tr, restart_every=every)
+    for k, R, Qacc, X in tr:
+        if k in points:
+            assert np.array_equal(Qacc, np.eye(12))
+            assert np.allclose(R, X @ X.T, rtol=0, atol=1e-14)
+    assert rel(out, oracle.ns_standard(X0, Q5[:1] * iters)) < 1e-12
 
 
 @pytest.mark.parametrize("shape", [(8, 24), (16, 16)])
