@@ -37,18 +37,23 @@ sys.path.insert(0, ROOT)
 import torch  # noqa: E402
 
 METRIC = "NS-orthogonalization ms/optimizer-step & effective TFLOP/s (% of bf16 peak)"
-# DRAM bytes (read + write) per product-kernel launch, keyed by (workload,
-# compute type).  bf16 Kimi-K2: averaged over the 45 launches of one step
-# (profiles/launches_kimi_k2_step.md).  fp32 dense: the three products of one
-# iteration captured on the 16-matrix set (profiles/gemm_tf32x3_kernel_dense16_fp32.md),
-# averaged (a step repeats them five times), and x4 for the 64-matrix set, whose
-# traffic grows with the matrix count.  Reset an entry to None whenever its
-# kernel changes until a new capture is taken.
-PRODUCT_TRAFFIC_PER_LAUNCH = {("kimi-k2", "bf16"): 18.89e9,
-                              ("dense16", "fp32"): 320.4e6, ("dense", "fp32"): 4 * 320.4e6}
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor rate on B200
 
-
+# Sources of each product kernel class: a DRAM-traffic figure holds only for
+# the kernel it was captured on, so each entry of MEASURED_TRAFFIC records the
+# hash of these files at capture time, and a changed kernel reports null.
+KERNEL_SOURCES = {
+    "tc_chain": ("gemm_chain.cu", "tc_common.cuh"),
+    "tc_product": ("gemm_tc2.cu", "gemm_tc.cu", "tc_common.cuh"),
+    "tc_product[symmetric]": ("gemm_tc2.cu", "gemm_tc.cu", "tc_common.cuh"),
+    "tc_product[3xtf32]": ("gemm_tf32.cu", "tc_common.cuh"),
+}
+# (workload, compute type, kernel class) -> (source hash, DRAM bytes read +
+# written per launch, averaged over the launches of one step, from an ncu
+# launch list of `python bench.py --workload <w> --compute <c> --steps 1
+# --warmup 1` with --metrics dram__bytes_read.sum,dram__bytes_write.sum).
+MEASURED_TRAFFIC: dict = {}
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
@@ -187,42 +192,76 @@ class ClockSampler:
                 "power_w_max": max(num(r[3]) for r in rows)}
 
 
-TF32_PER_BF16 = 1.1 / 2.25  # nominal dense TF32 : BF16 tensor rate on B200
-
-
-def roofline_from_profile(prof, peaks, peak_kind, workload=None, compute="bf16"):
-    fp32 = compute == "fp32"
-    gemm = [r for r in prof if r["kernel"].startswith("tc_product") and r["kernel"].endswith("[3xtf32]") == fp32]
-    if not gemm:
+def kernel_source_hash(kernel: str) -> str | None:
+    import hashlib
+    files = KERNEL_SOURCES.get(kernel)
+    if not files:
         return None
-    fl = sum(r["flops"] for r in gemm)
-    ms = sum(r["ms"] for r in gemm)
-    n = sum(r["launches"] for r in gemm)
-    bf16_peak = peaks["bf16_tflops_sustained"] if "bf16_tflops_sustained" in peaks else peaks["bf16_tflops"]
-    if fp32:
-        # three TF32 MMAs per product term (hi*hi, hi*lo, lo*hi): executed TF32 FLOP/s against
-        # the TF32 peak, i.e. the measured burst BF16 peak times the nominal TF32 : BF16 ratio
-        # (the fp32 steps run far below the power cap, at the maximum SM clock)
-        achieved = 3 * fl / (ms / 1e3) / 1e12
-        peak = round(peaks["bf16_tflops"] * TF32_PER_BF16, 1)
-        return {"bound": "tensor",
-                "kernel": "tcgen05 kind::tf32 3xTF32 product kernel (gemm_tf32x3_kernel), all launches of the step",
-                "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{peak_kind} bf16_tflops (burst) x {TF32_PER_BF16:.4f} (nominal TF32:BF16), "
-                               "achieved counts the three TF32 MMAs per product term",
-                "algorithmic_tflops": round(fl / (ms / 1e3) / 1e12, 1),
-                "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n,
-                "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get((workload, compute)),
-                "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per product launch (ncu)"}
-    achieved = fl / (ms / 1e3) / 1e12
-    return {"bound": "tensor",
-            "kernel": "tcgen05 product kernels (gemm_pair_kernel, gemm_kernel below 256 rows), all launches of the step",
-            "achieved": round(achieved, 1), "peak": bf16_peak, "unit": "TFLOP/s", "frac": round(achieved / bf16_peak, 4),
-            "peak_source": f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)",
-            "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
-            "per_launch_ms": round(ms / n, 4), "per_launch_flops": fl / n,
-            "traffic": PRODUCT_TRAFFIC_PER_LAUNCH.get((workload, compute)),
-            "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per product launch (ncu, one step)"}
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "newton_schulz_matrix_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload, compute, kernel):
+    """Captured DRAM bytes per launch, or None when there is no capture of the
+    current kernel source for this workload."""
+    e = MEASURED_TRAFFIC.get((workload, compute, kernel))
+    if e is None or e[0] != kernel_source_hash(kernel):
+        return None
+    return e[1]
+
+
+def roofline_from_profile(prof, peaks, peak_kind, workload=None, compute="fp16"):
+    """Roofline of the dominant product kernel class (the one with the most
+    device time), from the library's per-launch profile.
+
+    achieved = FLOPs the tensor cores execute in that class (whole tiles; the
+    upper-triangle tiles of symmetric products; three TF32 MMAs per 3xTF32
+    product) / its device time, against the tensor peak for its input type:
+    the sustained bf16 peak for 16-bit products (they run inside a seconds-long
+    stream of steps under the power cap; fp16 and bf16 share the kind::f16
+    rate), the burst bf16 peak x the nominal TF32:BF16 ratio for 3xTF32
+    (those steps run at the maximum clock).  The algorithmic rate (2 M N K per
+    product) is given beside it; every class is listed under by_kernel."""
+    fp32 = compute == "fp32"
+    bf16_sust = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tf32_peak = round(peaks["bf16_tflops"] * TF32_PER_BF16, 1)
+    hbm = peaks["hbm_gbs"]
+    rows = []
+    for r in prof:
+        k = r["kernel"]
+        if r["ms"] <= 0:
+            continue
+        sec = r["ms"] / 1e3
+        row = {"kernel": k, "launches": r["launches"], "ms": round(r["ms"], 4)}
+        if k.startswith("tc_product"):
+            peak = tf32_peak if k.endswith("[3xtf32]") else bf16_sust
+            ex = r.get("exec_flops", r["flops"])
+            row.update(bound="tensor", executed_tflops=round(ex / sec / 1e12, 1),
+                       algorithmic_tflops=round(r["flops"] / sec / 1e12, 1), peak=peak,
+                       frac=round(ex / sec / 1e12 / peak, 4), exec_flops_per_launch=ex / r["launches"])
+        elif r["bytes"] > 0:
+            row.update(bound="hbm", gbs=round(r["bytes"] / sec / 1e9, 1), peak=hbm,
+                       frac=round(r["bytes"] / sec / 1e9 / hbm, 4))
+        rows.append(row)
+    tensor = [x for x in rows if x.get("bound") == "tensor" and x["kernel"].endswith("[3xtf32]") == fp32]
+    if not tensor:
+        return None
+    dom = max(tensor, key=lambda x: x["ms"])
+    peak_source = (f"{peak_kind} bf16_tflops (burst) x {TF32_PER_BF16:.4f} (nominal TF32:BF16)" if fp32 else
+                   f"{peak_kind} bf16_tflops_sustained (kernel timed inside a long step)")
+    return {"bound": "tensor", "kernel": dom["kernel"],
+            "achieved": dom["executed_tflops"], "peak": dom["peak"], "unit": "TFLOP/s", "frac": dom["frac"],
+            "achieved_is": "executed tensor-core FLOPs / device time (CUDA events around each launch)",
+            "peak_source": peak_source, "algorithmic_tflops": dom["algorithmic_tflops"],
+            "per_launch_ms": round(dom["ms"] / dom["launches"], 4),
+            "per_launch_exec_flops": dom["exec_flops_per_launch"],
+            "traffic": measured_traffic(workload, compute, dom["kernel"]),
+            "traffic_note": "dram__bytes_read.sum + dram__bytes_write.sum per launch (ncu launch list of the "
+                            "same workload and kernel source); null when no capture of this source exists",
+            "by_kernel": rows}
 
 
 def cpu_baseline_sample(w, hp, budget_s=20.0):
@@ -378,7 +417,7 @@ def main():
     peaks, peak_kind = load_peaks()
     w, params, grads, moms = build_workload(args.workload, device)
     hp = dict(w.hp, mode=args.mode)
-    compute = hp.get("compute_dtype", "bf16")
+    compute = hp.get("compute_dtype", "fp16")
     if args.compute is not None:
         compute = args.compute
     ws_cap = int(args.workspace_gb * (1 << 30))
@@ -421,7 +460,6 @@ def main():
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(device)
-    nsm.muon_profile_begin()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -430,9 +468,24 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(device)
     barrier()
-    prof = nsm.muon_profile_end()
     clk = clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dist, device)
+    # the same steps again with every library launch bracketed by CUDA events on
+    # its stream: per-kernel device time for the roofline and the launch count
+    # (a separate pass, so the two events per launch stay out of the headline)
+    barrier()
+    torch.cuda.synchronize(device)
+    nsm.muon_profile_begin()
+    p0 = torch.cuda.Event(enable_timing=True)
+    p1 = torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(args.steps):
+        step()  # eager even under --graph: a replay makes no library calls to bracket
+    p1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    prof = nsm.muon_profile_end()
+    prof_ms = p0.elapsed_time(p1) / args.steps
     status = step.local.status.cpu() if args.sharded and step.local is not None else (
         torch.zeros(1, dtype=torch.int32) if args.sharded else step.status.cpu())
     value = whole_job_tflops(world, flops_step, ms)
@@ -521,6 +574,10 @@ def main():
             "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
             "scaling": "strong" if args.sharded else "weak",
             "vs_baseline": None, "dtype": {"bf16": "bf16", "fp16": "f16", "fp32": "f32"}[compute],
+            "dtype_note": (f"chain storage {compute} (X0, A, B or the Gram matrices between the products; "
+                           f"fp32 accumulation); parameters W and gradients G stay in their own types "
+                           f"({', '.join(sorted({str(p.dtype).replace('torch.', '') for p in params}))}), "
+                           "momentum fp32"),
             "data": "synthetic (seeded recipes of the workload; no datasets)",
             "config": dict(workload_config(w, params, hp["mode"], f"inputs larger than L2 ({resident / 2**30:.1f} GiB resident)"),
                            parallelism=(f"sharded over {world} ranks (owner broadcast)" if args.sharded
@@ -531,6 +588,7 @@ def main():
                       "source": peak_kind},
             "flops_per_step": flops_step,
             "clocks": clk, "e2e": e2e, "gpu_launches": launches_timed, "roofline": roof, "cpu_baseline": cpu,
+            "profiled_ms_per_step": round(prof_ms, 3),
             "kernels": [{k: (round(v, 4) if isinstance(v, float) else v) for k, v in r.items()} for r in prof],
             "status_nonzero": int((status != 0).sum()),
         }

@@ -19,7 +19,7 @@
  *     use: the SM count, shared-memory opt-ins, how many CTA pairs fit).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream).  They take no lock on the launch path; the opt-in
- *     profiler and the allocation-free entry point's one-time scratch lookup
+ *     profiler and the allocation-free entry point's scratch lookup
  *     take a mutex.  The return value reports argument
  *     and launch errors only (MUON_OK, MUON_ERR_*).  Conditions found on the
  *     device are OR-ed into the optional per-matrix status words (device int
@@ -53,8 +53,9 @@ typedef enum { MUON_BF16 = 0, MUON_FP16 = 1, MUON_FP32 = 2 } muon_dtype;
  *   STANDARD         X <- a X + (b A + c A^2) X, A = X X^T, per iteration
  *   GRAM             naive Gram form: R = X0 X0^T; Q_k = a I + b R + c R^2;
  *                    Q_acc <- Q_k Q_acc; R <- Q_k R Q_k; X = Q_acc X0
- *   GRAM_STABILIZED  Gram form restarted once after iteration restart_after:
- *                    X0 <- Q_acc X0, R <- X0 X0^T, Q_acc <- I */
+ *   GRAM_STABILIZED  Gram form restarted after iteration restart_after (and,
+ *                    if restart_every > 0, every restart_every iterations
+ *                    after it): X0 <- Q_acc X0, R <- X0 X0^T, Q_acc <- I */
 typedef enum { MUON_NS_STANDARD = 0, MUON_NS_GRAM = 1, MUON_NS_GRAM_STABILIZED = 2 } muon_ns_mode;
 
 enum {
@@ -75,6 +76,9 @@ enum {
  *   mode           muon_ns_mode
  *   restart_after  GRAM_STABILIZED only: iteration after which the Gram
  *                  matrix is rebuilt (1 <= restart_after < iters; 2 in [GramNS])
+ *   restart_every  GRAM_STABILIZED only: 0 = rebuild once; e > 0 = also after
+ *                  iterations restart_after + e, + 2e, ... before the last
+ *                  (the periodic reading of [GramNS]'s "re-initialise")
  *   eps            X0 = U / (||U||_F + eps)  [Moonlight, NS section; listing eps]
  *   compute_dtype  MUON_BF16 or MUON_FP16: tcgen05 tensor cores, fp32
  *                  accumulate, 16-bit storage of X, A, B between the products
@@ -94,6 +98,7 @@ typedef struct {
   float eps;
   int compute_dtype;
   int gram_dtype;
+  int restart_every;
 } muon_ns_params;
 
 /* One group of `count` parameters that share storage shape rows x cols.
@@ -161,12 +166,15 @@ MUON_API int muon_ns_batched(void* const* X, int count, int rows, int cols, int 
  * rejected with MUON_ERR_WORKSPACE; larger counts of fitting matrices are
  * processed in chunks.  Results equal muon_ns_batched's.
  *
- * The first call on a device looks up the array's device address with that
- * device current (cudaGetSymbolAddress) and caches it: make that first call
- * before any stream capture.  Every call uses the same array, which keeps
- * the previous call's contents (the call resets what must start at zero):
- * calls that can overlap on the GPU (other streams, other host threads)
- * race on it and must be serialised by the caller, e.g. on one stream. */
+ * A call outside a stream capture looks up the array's device address on
+ * the current device (cudaGetSymbolAddress) and remembers it; a call on a
+ * capturing stream uses the address remembered by the last uncaptured call on
+ * that device (none: MUON_ERR_CUDA), so make one uncaptured call before
+ * capturing, and again after a cudaDeviceReset.  Every call uses the same
+ * array, which keeps the previous call's contents (the call resets what must
+ * start at zero): calls that can overlap on the GPU (other streams, other
+ * host threads) race on it and must be serialised by the caller, e.g. on one
+ * stream. */
 #define MUON_NOALLOC_SCRATCH_BYTES (64u << 20)
 MUON_API int muon_ns_batched_noalloc(void* const* X, int count, int rows, int cols, int dtype,
                                      const muon_ns_params* ns, int* status_per_matrix, void* stream);
@@ -181,14 +189,21 @@ MUON_API double muon_ns_flops(int rows, int cols, const muon_ns_params* ns);
  * library keeps between calls, and only while profiling is on.
  * muon_profile_end synchronises on those events and fills up to max_entries
  * rows, one per kernel kind that ran: its name, launch count, summed device
- * time, and the algorithmic FLOPs and bytes of those launches (products count
- * 2 * M * N * K, the full product even where only a triangle is computed).
+ * time, and for those launches
+ *   flops       algorithmic FLOPs: every product 2 * M * N * K, the full
+ *               product even where only a triangle is computed [GramNS cost list]
+ *   exec_flops  FLOPs the kernels execute: tensor-core MMAs over whole tiles
+ *               (zero padding included), only the tiles of a symmetric
+ *               product's upper triangle, three TF32 MMAs per 3xTF32 product;
+ *               equal to flops for the other kernels
+ *   bytes       algorithmic bytes (each operand read once, result written once)
  * Returns the number of rows written, or a MUON_ERR_* code. */
 typedef struct {
   const char* kernel;
   int launches;
   double ms;
   double flops;
+  double exec_flops;
   double bytes;
 } muon_profile_entry;
 MUON_API int muon_profile_begin(void);

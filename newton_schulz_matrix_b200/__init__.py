@@ -50,7 +50,7 @@ class MuonError(RuntimeError):
 class _NSParams(ctypes.Structure):
     _fields_ = [("iters", ctypes.c_int), ("coeffs", ctypes.POINTER(ctypes.c_float)), ("mode", ctypes.c_int),
                 ("restart_after", ctypes.c_int), ("eps", ctypes.c_float), ("compute_dtype", ctypes.c_int),
-                ("gram_dtype", ctypes.c_int)]
+                ("gram_dtype", ctypes.c_int), ("restart_every", ctypes.c_int)]
 
 
 class _Group(ctypes.Structure):
@@ -67,7 +67,7 @@ class _HParams(ctypes.Structure):
 
 class _ProfEntry(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_char_p), ("launches", ctypes.c_int), ("ms", ctypes.c_double),
-                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
+                ("flops", ctypes.c_double), ("exec_flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 def library_path() -> str:
@@ -128,11 +128,12 @@ def _code(v, names) -> int:
     return names[v] if isinstance(v, str) else int(v)
 
 
-def _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype):
+def _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype, restart_every=0):
     flat = [float(x) for abc in coeffs for x in abc]
     arr = (ctypes.c_float * len(flat))(*flat)
     p = _NSParams(len(flat) // 3, ctypes.cast(arr, ctypes.POINTER(ctypes.c_float)), _code(mode, _MODE_NAMES),
-                  int(restart_after), float(eps), _code(compute_dtype, _DT_NAMES), _code(gram_dtype, _DT_NAMES))
+                  int(restart_after), float(eps), _code(compute_dtype, _DT_NAMES), _code(gram_dtype, _DT_NAMES),
+                  int(restart_every))
     return p, arr
 
 
@@ -196,24 +197,25 @@ def muon_status_string(code: int) -> str:
     return load_library().muon_status_string(int(code)).decode()
 
 
-def muon_ns_flops(rows: int, cols: int, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2) -> float:
-    ns, _arr = _ns_params(coeffs, mode, restart_after, 1e-7, BF16, FP16)
+def muon_ns_flops(rows: int, cols: int, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2,
+                  restart_every=0) -> float:
+    ns, _arr = _ns_params(coeffs, mode, restart_after, 1e-7, BF16, FP16, restart_every)
     return load_library().muon_ns_flops(rows, cols, ctypes.byref(ns))
 
 
 def _step_args(params, grads, moms, lr, momentum, nesterov, weight_decay, scale_coef, eps, coeffs, mode,
-               restart_after, compute_dtype, gram_dtype):
+               restart_after, compute_dtype, gram_dtype, restart_every=0):
     if not (len(params) == len(grads) == len(moms)) or len(params) == 0:
         raise MuonError("params, grads and moms must be non-empty lists of equal length")
     groups, ng, keep, order = _build_groups(params, grads, moms)
-    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype, restart_every)
     hp = _hparams(lr, momentum, weight_decay, scale_coef, nesterov, ns)
     return groups, ng, hp, (keep, arr), order
 
 
 _STEP_DEFAULTS = dict(lr=0.02, momentum=0.95, nesterov=True, weight_decay=0.1, scale_coef=0.2, eps=1e-7,
-                      coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2, compute_dtype="bf16",
-                      gram_dtype="fp16")
+                      coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2, compute_dtype="fp16",
+                      gram_dtype="fp16", restart_every=0)
 
 
 def muon_workspace_size(params, grads, moms, **hp) -> int:
@@ -235,7 +237,12 @@ def muon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor], mom
 
     Keyword hyper-parameters (defaults: lr 0.02, momentum 0.95, nesterov True,
     weight_decay 0.1, scale_coef 0.2, eps 1e-7, five quintic iterations,
-    mode "standard", restart_after 2, compute_dtype "bf16", gram_dtype "fp16").
+    mode "standard", restart_after 2, restart_every 0, compute_dtype "fp16",
+    gram_dtype "fp16").
+    ``compute_dtype`` is the storage type of the chain between the products
+    (W and G keep their own types): "fp16" stores X0 = U / (||U|| + eps) and
+    every product in binary16, "bf16" stores the raw U and the products in
+    bfloat16 (8 x coarser), "fp32" runs 3xTF32 products.
     ``workspace`` is a CUDA uint8 tensor (allocated when None); ``status``, if
     given, is an int32 CUDA tensor with one word per parameter (in the order of
     ``params``) and receives the MUON_STATUS_* bits.
@@ -262,22 +269,25 @@ def muon_step(params: Sequence[torch.Tensor], grads: Sequence[torch.Tensor], mom
 
 
 def muon_ns_workspace_size(count: int, rows: int, cols: int, coeffs=(QUINTIC,) * 5, mode="standard",
-                           restart_after=2, eps=1e-7, compute_dtype="bf16", gram_dtype="fp16") -> int:
-    ns, _arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+                           restart_after=2, eps=1e-7, compute_dtype="fp16", gram_dtype="fp16",
+                           restart_every=0) -> int:
+    ns, _arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype, restart_every)
     return int(load_library().muon_ns_workspace_size(count, rows, cols, ctypes.byref(ns)))
 
 
 def muon_ns_batched(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2,
                     eps=1e-7, compute_dtype=None, gram_dtype="fp16", workspace: torch.Tensor | None = None,
-                    status: torch.Tensor | None = None, stream=None) -> None:
+                    status: torch.Tensor | None = None, stream=None, restart_every=0) -> None:
     """Orthogonalise same-shape matrices in place (result has each input's shape).
 
     ``compute_dtype`` is the storage type of the chain: None picks "fp32" for
-    fp32 inputs and "bf16" otherwise; "fp16" is also accepted.  fp32 chains run
+    fp32 inputs and "fp16" otherwise; "bf16" is also accepted.  fp32 chains run
     3xTF32 tensor-core products when the short side is at least 256, and a
     single fused launch per call for matrices small enough for one block's
     shared memory.  ``gram_dtype`` is the 16-bit type of the Gram chains.
     ``status``, if given, is an int32 CUDA tensor with one word per matrix.
+    ``restart_every`` > 0 repeats the stabilised form's restart every that many
+    iterations after ``restart_after``.
     """
     lib = load_library()
     if len(X) == 0:
@@ -289,8 +299,8 @@ def muon_ns_batched(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5, mode="s
     rows, cols = X[0].shape
     dt = _dtype_code(X[0].dtype)
     if compute_dtype is None:
-        compute_dtype = "fp32" if dt == FP32 else "bf16"
-    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+        compute_dtype = "fp32" if dt == FP32 else "fp16"
+    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype, restart_every)
     need = int(lib.muon_ns_workspace_size(len(X), rows, cols, ctypes.byref(ns)))
     if need == 0:
         raise MuonError("invalid arguments (workspace query returned 0)")
@@ -310,13 +320,15 @@ def muon_profile_begin() -> None:
 
 
 def muon_profile_end() -> list[dict]:
-    """Stop profiling; per kernel kind: launches, device ms, algorithmic FLOPs and bytes."""
+    """Stop profiling; per kernel kind: launches, device ms, algorithmic FLOPs,
+    executed FLOPs (whole tensor-core tiles, triangles only for symmetric
+    products, three MMAs per 3xTF32 product) and algorithmic bytes."""
     rows = (_ProfEntry * 16)()
     n = load_library().muon_profile_end(rows, 16)
     if n < 0:
         _raise(n, "muon_profile_end")
-    return [dict(kernel=r.kernel.decode(), launches=r.launches, ms=r.ms, flops=r.flops, bytes=r.bytes)
-            for r in rows[:n]]
+    return [dict(kernel=r.kernel.decode(), launches=r.launches, ms=r.ms, flops=r.flops, exec_flops=r.exec_flops,
+                 bytes=r.bytes) for r in rows[:n]]
 
 
 class MuonStep:
@@ -378,7 +390,7 @@ class MuonStep:
 
 def muon_ns_batched_noalloc(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5, mode="standard", restart_after=2,
                             eps=1e-7, compute_dtype=None, gram_dtype="fp16", status: torch.Tensor | None = None,
-                            stream=None) -> None:
+                            stream=None, restart_every=0) -> None:
     """muon_ns_batched with the library's fixed device scratch instead of a
     workspace: for callers that cannot allocate device memory at this point
     (their allocator owns the GPU, or allocation is forbidden after start-up).
@@ -395,8 +407,8 @@ def muon_ns_batched_noalloc(X: Sequence[torch.Tensor], *, coeffs=(QUINTIC,) * 5,
     rows, cols = X[0].shape
     dt = _dtype_code(X[0].dtype)
     if compute_dtype is None:
-        compute_dtype = "fp32" if dt == FP32 else "bf16"
-    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype)
+        compute_dtype = "fp32" if dt == FP32 else "fp16"
+    ns, arr = _ns_params(coeffs, mode, restart_after, eps, compute_dtype, gram_dtype, restart_every)
     ptrs = (ctypes.c_void_p * len(X))(*[t.data_ptr() for t in X])
     rc = lib.muon_ns_batched_noalloc(ptrs, len(X), rows, cols, dt, ctypes.byref(ns),
                                      ctypes.c_void_p(status.data_ptr() if status is not None else 0),

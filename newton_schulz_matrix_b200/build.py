@@ -18,7 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmuon.so")
-SOURCES = ["api.cu", "elementwise.cu", "gemm_simt.cu", "gemm_tc.cu", "gemm_tc2.cu", "gemm_tf32.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "elementwise.cu", "gemm_chain.cu", "gemm_simt.cu", "gemm_tc.cu", "gemm_tc2.cu", "gemm_tf32.cu",
+           "noalloc.cu"]
 HEADERS = ["common.cuh", "internal.h", "tc_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -12,7 +12,7 @@
 //
 // The iteration order follows the "Gram Newton-Schulz" write-up (standard
 // form: A = X X^T, B = b A + c A^2, X = a X + B X; Gram form: iterate on
-// R = X X^T, accumulate Q_acc = Q_k ... Q_1, restart once in the stabilised
+// R = X X^T, accumulate Q_acc = Q_k ... Q_1, restart in the stabilised
 // variant) and the optimizer step of "Moonlight 16B Guide" (box steps 1-4).
 #include <stdint.h>
 #include <stdlib.h>
@@ -37,16 +37,18 @@ inline int round8(int v) { return (v + 7) / 8 * 8; }
 
 // ------------------------------------------------------------------ profiler
 enum ProfKind {
-  kProfPack, kProfNorm, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfFusedSmall, kProfTf32, kProfKinds
+  kProfPack, kProfNorm, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfFusedSmall, kProfTf32, kProfChain,
+  kProfStatus, kProfKinds
 };
-// product kinds cover both tensor-core kernels (gemm_pair_kernel for M >= 256, gemm_kernel below)
+// product kinds cover both tensor-core kernels (gemm_pair_kernel for M >= 256, gemm_kernel below);
+// tc_chain is a whole chain in one launch (gemm_chain_kernel)
 const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "tc_product[symmetric]", "tc_product",
                                             "gemm_simt_kernel", "unpack_kernel", "ns_fused_small_kernel",
-                                            "tc_product[3xtf32]"};
+                                            "tc_product[3xtf32]", "tc_chain", "status_or_kernel"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
-  double flops, bytes;
+  double flops, exec_flops, bytes;
 };
 struct Profiler {
   bool on = false;
@@ -62,10 +64,11 @@ struct ProfScope {
   ProfRec rec{};
   bool active = false;
   cudaStream_t s;
-  ProfScope(int kind, double flops, double bytes, cudaStream_t st) : s(st) {
+  ProfScope(int kind, double flops, double bytes, cudaStream_t st, double exec_flops = -1.0) : s(st) {
     Profiler& P = profiler();
     if (!P.on) return;
     rec.kind = kind; rec.flops = flops; rec.bytes = bytes;
+    rec.exec_flops = exec_flops < 0.0 ? flops : exec_flops;
     if (cudaEventCreate(&rec.a) != cudaSuccess) return;
     if (cudaEventCreate(&rec.b) != cudaSuccess) { cudaEventDestroy(rec.a); return; }
     cudaEventRecord(rec.a, s);
@@ -95,6 +98,9 @@ struct Layout {       // per-chunk workspace layout for a batch
   int x_es, g_es;     // element sizes of X and Gram buffers
   int n_sq;           // number of n x n buffers
   int tiles;          // pack tiles per matrix (sums-of-squares partials)
+  int n_counters;     // tile-scheduler words: one per product launch of the chain
+  size_t head;        // error word + counters, zeroed at the start of each chunk
+                      // (followed by the chain launches' done counters: n_counters per matrix)
   size_t per_matrix;  // bytes per matrix (all buffers)
   size_t fixed;       // bytes independent of the chunk size
 };
@@ -103,6 +109,7 @@ bool ns_params_ok(const muon_ns_params* ns) {
   if (!ns || ns->iters < 1 || ns->iters > 1000 || !ns->coeffs) return false;
   if (ns->mode < MUON_NS_STANDARD || ns->mode > MUON_NS_GRAM_STABILIZED) return false;
   if (ns->mode == MUON_NS_GRAM_STABILIZED && (ns->restart_after < 1 || ns->restart_after >= ns->iters)) return false;
+  if (ns->restart_every < 0) return false;
   if (!(ns->eps >= 0.f) || !std::isfinite(ns->eps)) return false;
   if (ns->compute_dtype < MUON_BF16 || ns->compute_dtype > MUON_FP32) return false;
   if (ns->mode != MUON_NS_STANDARD && ns->compute_dtype != MUON_FP32 && ns->gram_dtype != MUON_BF16 &&
@@ -124,9 +131,14 @@ Layout make_layout(int n, int m, const muon_ns_params* ns) {
   L.g_es = ns->compute_dtype == MUON_FP32 ? 4 : 2;
   L.n_sq = ns->mode == MUON_NS_STANDARD ? 2 : 5;
   L.tiles = pack_tiles(n, m);
+  // at most 6 product launches per iteration (Gram form: R^2, Q Q_acc, T, R or a
+  // restart pair) plus R0 and the final apply
+  L.n_counters = 6 * ns->iters + 8;
+  L.head = align_up(kAlign + (size_t)L.n_counters * 4, kAlign);
   // buffers: 2 X, n_sq Gram-sized, partials, inv (each 256-byte aligned per chunk)
-  L.per_matrix = 2 * (size_t)n * L.ld_m * L.x_es + (size_t)L.n_sq * n * L.ld_n * L.g_es + (size_t)L.tiles * 4 + 4;
-  L.fixed = kAlign * (2 + L.n_sq + 2 + 1) + kAlign;  // alignment slack + error word
+  L.per_matrix = 2 * (size_t)n * L.ld_m * L.x_es + (size_t)L.n_sq * n * L.ld_n * L.g_es + (size_t)L.tiles * 4 + 4 +
+                 (size_t)L.n_counters * 4;
+  L.fixed = kAlign * (2 + L.n_sq + 3) + kAlign + L.head;  // alignment slack + error word and counters
   return L;
 }
 
@@ -138,6 +150,9 @@ struct Bufs {
   float* partials;
   float* inv;
   int* err;
+  int* counters;      // L.n_counters words after the error word's 256-byte slot
+  int* done;          // chunk * L.n_counters words: per product and matrix, for chain launches
+  size_t zero_bytes;  // from err through done: zeroed at the start of the chunk
   long long x_bs, s_bs;
 };
 
@@ -145,7 +160,11 @@ Bufs carve(const Layout& L, int chunk, void* ws) {
   Bufs B{};
   char* p = reinterpret_cast<char*>(align_up(reinterpret_cast<uintptr_t>(ws), kAlign));
   B.err = reinterpret_cast<int*>(p);
-  p += kAlign;
+  B.counters = reinterpret_cast<int*>(p + kAlign);
+  p += L.head;
+  B.done = reinterpret_cast<int*>(p);
+  p += align_up((size_t)chunk * L.n_counters * 4, kAlign);
+  B.zero_bytes = L.head + align_up((size_t)chunk * L.n_counters * 4, kAlign);
   B.x_bs = (long long)L.n * L.ld_m;
   B.s_bs = (long long)L.n * L.ld_n;
   for (int i = 0; i < 2; ++i) {
@@ -185,6 +204,10 @@ struct Ctx {
   int compute;   // MUON_BF16 / MUON_FP16 / MUON_FP32
   cudaStream_t s;
   int* err;
+  int* counters;       // zeroed tile-scheduler words, one per product launch
+  int n_counters;
+  int* used;           // how many of them the chain has taken so far
+  std::vector<GemmDesc>* record = nullptr;  // chain mode: collect the products instead of launching them
 };
 
 // fp32 products with 256 or more rows run as 3xTF32 on the tensor cores;
@@ -199,19 +222,26 @@ bool fp32_tensor_cores() {
 
 int gemm(const Ctx& c, GemmDesc g) {
   g.err = c.err;
+  if (c.record != nullptr) {
+    c.record->push_back(g);
+    return 0;
+  }
+  if (*c.used >= c.n_counters) return (int)cudaErrorInvalidValue;
+  g.tile_counter = c.counters + (*c.used)++;
   const double flops = 2.0 * g.M * g.N * (double)g.K * g.batch;
   const int es = dtype_size(g.in_dtype);
   const double bytes = ((double)g.M * g.K * es + (double)g.N * g.K * es + (double)g.M * g.N * dtype_size(g.d_dtype) +
                         (g.C ? (double)g.M * g.N * dtype_size(g.c_dtype) : 0.0)) * g.batch;
+  const bool prof = profiler().on;
   if (c.compute == MUON_FP32) {
     if (g.M >= 256 && fp32_tensor_cores()) {
-      ProfScope ps(kProfTf32, flops, bytes, c.s);
+      ProfScope ps(kProfTf32, flops, bytes, c.s, prof ? gemm_tf32x3_exec_flops(g) : 0.0);
       return gemm_tf32x3(g, c.s);
     }
     ProfScope ps(kProfGemmSimt, flops, bytes, c.s);
     return gemm_simt(g, c.s);
   }
-  ProfScope ps(g.symmetric ? kProfSyrkTc : kProfGemmTc, flops, bytes, c.s);
+  ProfScope ps(g.symmetric ? kProfSyrkTc : kProfGemmTc, flops, bytes, c.s, prof ? gemm_tc_exec_flops(g) : 0.0);
   return gemm_tc(g, c.s);
 }
 
@@ -232,12 +262,30 @@ GemmDesc desc(int M, int N, int K, int batch) {
 // the raw U (bf16's range holds any gradient) and applies f = 1/(||U||+eps)
 // inside the first products' epilogues; an fp16 chain receives X0 = f U
 // already normalised (`prescaled`), rounded once from fp32 to fp16.
+// Whether the stabilised Gram chain restarts after iteration k (1-based).
+bool restart_at(const muon_ns_params* ns, int k) {
+  if (ns->mode != MUON_NS_GRAM_STABILIZED || k >= ns->iters || k < ns->restart_after) return false;
+  if (k == ns->restart_after) return true;
+  return ns->restart_every > 0 && (k - ns->restart_after) % ns->restart_every == 0;
+}
+
 int chain_dtype(const muon_ns_params* ns) {
   if (ns->compute_dtype == MUON_FP32) return MUON_FP32;
   return ns->mode == MUON_NS_STANDARD ? ns->compute_dtype : ns->gram_dtype;
 }
 
 double flops_of(int rows, int cols, const muon_ns_params* ns);  // algorithmic FLOPs of one matrix's chain
+
+// 16-bit chains of a Muon step whose last product runs on the paired-CTA
+// kernel write the update from that product's epilogue (no unpack pass, no X
+// round trip through memory); MUON_FUSED_UPDATE=0 keeps the separate pass.
+bool fused_update_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("MUON_FUSED_UPDATE");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 // fp32 chains whose matrices fit in one CTA's shared memory run as a single
 // fused launch (one CTA per matrix); MUON_FUSED_SMALL=0 keeps the chained
@@ -262,14 +310,18 @@ int run_fused_small(const Ctx& c, const Layout& L, const Bufs& B, int chunk, con
   a.inv = B.inv; a.raw = prescaled ? 0 : 1;
   a.mode = ns->mode == MUON_NS_STANDARD ? 0 : 1;
   a.restart_after = ns->mode == MUON_NS_GRAM_STABILIZED ? ns->restart_after : 0;
+  a.restart_every = ns->mode == MUON_NS_GRAM_STABILIZED ? ns->restart_every : 0;
   a.iters = ns->iters;
   for (int i = 0; i < 3 * ns->iters; ++i) a.coeffs[i] = ns->coeffs[i];
   ProfScope ps(kProfFusedSmall, flops_of(L.n, L.m, ns) * chunk, 2.0 * chunk * L.n * L.m * 4, c.s);
   return launch_fused_small(a, c.s);
 }
 
+// `update` (may be null): the chain's last product writes the Muon update
+// into W through these slots instead of storing O (the result X is then not
+// written; see run_batches).
 int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns, bool prescaled,
-              int* out_x, int* out_dtype) {
+              int* out_x, int* out_dtype, const UpdateSlots* update = nullptr) {
   if (use_fused_small(L, ns)) {
     *out_x = 0;
     *out_dtype = MUON_FP32;
@@ -322,6 +374,7 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
       g.C = B.X[cur]; g.ldc = L.ld_m; g.c_bs = B.x_bs; g.c_dtype = xdt;
       g.c_acc = coefB; g.c_in = a;
       g.scale = B.inv; g.scale_pow = first ? 1 : 0;
+      if (k == K - 1) g.update = update;
       if ((rc = gemm(c, g))) return rc;
       cur = 1 - cur;
     }
@@ -330,7 +383,6 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
   }
 
   // ---------------------------------------------------------------- Gram forms
-  const bool stabilized = ns->mode == MUON_NS_GRAM_STABILIZED;
   int x0 = start;          // X buffer holding the matrix the Gram iteration applies to
   bool x0_raw = raw;       // still the unnormalised packed U (scale by inv on use)
   void* R = B.S[0];
@@ -355,8 +407,9 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
     g.in_dtype = gdt;
     g.D = D; g.ldd = L.ld_n; g.d_bs = B.s_bs; g.d_dtype = ddt;
   };
-  auto apply = [&](int x_out) -> int {  // X[x_out] = f Q_acc X0
+  auto apply = [&](int x_out, const UpdateSlots* upd) -> int {  // X[x_out] = f Q_acc X0
     GemmDesc g = desc(n, m, n, chunk);
+    g.update = upd;
     g.A = Qbuf[q_acc]; g.lda = L.ld_n; g.a_bs = B.s_bs;
     g.B = B.X[x0]; g.ldb = L.ld_m; g.b_bs = B.x_bs; g.b_kmajor = 0;
     g.in_dtype = xdt;
@@ -369,7 +422,7 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
   for (int k = 1; k <= K; ++k) {
     const float a = ns->coeffs[3 * (k - 1)], bb = ns->coeffs[3 * (k - 1) + 1], cc = ns->coeffs[3 * (k - 1) + 2];
     const bool last = k == K;
-    const bool restart = stabilized && k == ns->restart_after && !last;
+    const bool restart = restart_at(ns, k);
     const bool to_apply = last || restart;
     // Q = a I + b R + c R R, into a slot that is not Q_acc
     int qi = 0;
@@ -399,7 +452,7 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
     if (last) break;
     if (restart) {
       const int x_new = 1 - x0;
-      if ((rc = apply(x_new))) return rc;
+      if ((rc = apply(x_new, nullptr))) return rc;
       x0 = x_new;
       x0_raw = false;
       if ((rc = gram_of_x(false))) return rc;
@@ -420,8 +473,61 @@ int run_chain(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muo
     }
   }
   const int x_out = 1 - x0;
-  if ((rc = apply(x_out))) return rc;
+  if ((rc = apply(x_out, update))) return rc;
   *out_x = x_out;
+  return 0;
+}
+
+// Host-side slot table of the fused update (about 7 KB): one per host thread,
+// reused for every chunk; its contents are copied into the kernel parameters
+// at launch, so reuse after the launch call is safe.
+UpdateSlots& slots_storage() {
+  thread_local UpdateSlots slots;
+  return slots;
+}
+
+// 16-bit chains whose products all run on the paired-CTA kernel go out as
+// one persistent launch per (up to 24) products, with per-matrix dependency
+// counters in place of launch boundaries; MUON_CHAIN=0 launches every
+// product separately.
+bool chain_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("MUON_CHAIN");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// run_chain in one of two ways: product by product, or (chain mode) the same
+// products recorded and then launched as whole-chain segments.
+int run_chain_launch(const Ctx& c, const Layout& L, const Bufs& B, int chunk, const muon_ns_params* ns,
+                     bool prescaled, int* out_x, int* out_dtype, const UpdateSlots* update) {
+  const bool chain = chain_enabled() && ns->compute_dtype != MUON_FP32 && gemm_tc_paired(L.n);
+  if (!chain) return run_chain(c, L, B, chunk, ns, prescaled, out_x, out_dtype, update);
+  std::vector<GemmDesc> prods;
+  Ctx rc = c;
+  rc.record = &prods;
+  int rv = run_chain(rc, L, B, chunk, ns, prescaled, out_x, out_dtype, update);
+  if (rv) return rv;
+  const bool prof = profiler().on;
+  for (size_t first = 0; first < prods.size(); first += kChainMaxProducts) {
+    const int n = (int)std::min<size_t>(kChainMaxProducts, prods.size() - first);
+    if (*c.used >= c.n_counters) return (int)cudaErrorInvalidValue;
+    int* counter = c.counters + (*c.used)++;
+    double flops = 0.0, exec = 0.0, bytes = 0.0;
+    if (prof) {
+      for (int i = 0; i < n; ++i) {
+        const GemmDesc& g = prods[first + i];
+        flops += 2.0 * g.M * g.N * (double)g.K * g.batch;
+        exec += gemm_tc_exec_flops(g);
+        bytes += ((double)g.M * g.K * 2 + (double)g.N * g.K * 2 + (double)g.M * g.N * 2 +
+                  (g.C ? (double)g.M * g.N * 2 : 0.0)) * g.batch;
+      }
+    }
+    ProfScope ps(kProfChain, flops, bytes, c.s, exec);
+    rv = gemm_chain(prods.data() + first, n, counter, B.done + first * (size_t)chunk, c.err, c.s);
+    if (rv) return rv;
+  }
   return 0;
 }
 
@@ -440,14 +546,16 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
   for (const Batch& bt : batches) {
     const Layout L = make_layout(bt.n, bt.m, ns);
     if (ws_bytes < chunk_bytes(L, 1)) return MUON_ERR_WORKSPACE;
-    const int chunk_cap = (int)std::min<size_t>((size_t)bt.total, (ws_bytes - L.fixed) / L.per_matrix);
+    const bool fuse = update && ns->compute_dtype != MUON_FP32 && fused_update_enabled() && gemm_tc_paired(L.n);
+    int chunk_cap = (int)std::min<size_t>((size_t)bt.total, (ws_bytes - L.fixed) / L.per_matrix);
+    if (fuse) chunk_cap = std::min(chunk_cap, UpdateSlots::kMax);
     // slots are assigned in segment order; walk them chunk by chunk
     int seg_i = 0, seg_off = 0;
     int done = 0;
     while (done < bt.total) {
       const int chunk = std::min(chunk_cap, bt.total - done);
       const Bufs B = carve(L, chunk, ws);
-      if (cudaMemsetAsync(B.err, 0, sizeof(int), s) != cudaSuccess) return MUON_ERR_CUDA;
+      if (cudaMemsetAsync(B.err, 0, B.zero_bytes, s) != cudaSuccess) return MUON_ERR_CUDA;
       // pieces of segments covering slots [done, done + chunk)
       struct Piece { int group, first, count, slot; };
       std::vector<Piece> pieces;
@@ -508,9 +616,33 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
       }
       if (prescale) launch_pieces(2);
       if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
-      Ctx ctx{ns->compute_dtype, s, B.err};
+      int used = 0;
+      Ctx ctx{ns->compute_dtype, s, B.err, B.counters, L.n_counters, &used};
       int xi = 0, out_dt = pack_dt;
-      if (run_chain(ctx, L, B, chunk, ns, prescale, &xi, &out_dt) != 0) return MUON_ERR_CUDA;
+      if (fuse) {
+        UpdateSlots& us = slots_storage();
+        us.decay = 1.f - lr * wd;
+        us.step = lr * scale_coef * std::sqrt((float)bt.m);  // max(rows, cols) = m for every matrix of the batch
+        us.status = status;
+        for (const Piece& pc : pieces) {
+          const SrcView& v = views[pc.group];
+          for (int i = 0; i < pc.count; ++i) {
+            us.w[pc.slot + i] = v.dst[pc.first + i];
+            us.status_idx[pc.slot + i] = (int)(first_index[pc.group] + pc.first + i);
+            us.kind[pc.slot + i] = (unsigned char)((v.rows > v.cols ? 1 : 0) | (v.dst_dtype << 1));
+          }
+        }
+        if (run_chain_launch(ctx, L, B, chunk, ns, prescale, &xi, &out_dt, &us) != 0) return MUON_ERR_CUDA;
+        if (status)
+          for (const Piece& pc : pieces) {
+            ProfScope ps(kProfStatus, 0.0, pc.count * 8.0, s);
+            launch_status_or(status + first_index[pc.group] + pc.first, pc.count, B.err, s);
+          }
+        if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
+        done += chunk;
+        continue;
+      }
+      if (run_chain_launch(ctx, L, B, chunk, ns, prescale, &xi, &out_dt, nullptr) != 0) return MUON_ERR_CUDA;
       for (const Piece& pc : pieces) {
         const SrcView& v = views[pc.group];
         SegmentPtrs ptrs;
@@ -593,7 +725,7 @@ double flops_of(int rows, int cols, const muon_ns_params* ns) {
     if (!fresh) total += cube;
     fresh = false;
     if (k == K) break;
-    if (ns->mode == MUON_NS_GRAM_STABILIZED && k == ns->restart_after) {
+    if (restart_at(ns, k)) {
       total += 2 * sq;
       fresh = true;
     } else {
@@ -688,7 +820,7 @@ int muon_profile_end(muon_profile_entry* out, int max_entries) {
   std::lock_guard<std::mutex> g(P.mu);
   P.on = false;
   muon_profile_entry acc[kProfKinds];
-  for (int k = 0; k < kProfKinds; ++k) acc[k] = muon_profile_entry{kProfNames[k], 0, 0.0, 0.0, 0.0};
+  for (int k = 0; k < kProfKinds; ++k) acc[k] = muon_profile_entry{kProfNames[k], 0, 0.0, 0.0, 0.0, 0.0};
   int rc = MUON_OK;
   for (auto& r : P.recs) {
     float ms = 0.f;
@@ -696,6 +828,7 @@ int muon_profile_end(muon_profile_entry* out, int max_entries) {
     acc[r.kind].launches += 1;
     acc[r.kind].ms += ms;
     acc[r.kind].flops += r.flops;
+    acc[r.kind].exec_flops += r.exec_flops;
     acc[r.kind].bytes += r.bytes;
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);

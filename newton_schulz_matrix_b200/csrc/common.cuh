@@ -46,6 +46,14 @@ __device__ __forceinline__ float matrix_scale(const float* scale, int pow, int b
   return pow == 2 ? s * s : s;
 }
 
+// The decoupled-weight-decay update of one element, W <- (1 - lr wd) W - step O
+// ("Moonlight 16B Guide", Innovation 1 and box step 4), with its rounding fixed:
+// decay * w rounded once, then one fused multiply-add.  Every kernel that
+// writes W uses this, so the results do not depend on which one ran.
+__device__ __forceinline__ float weight_update(float w, float o, float decay, float step) {
+  return __fmaf_rn(-step, o, __fmul_rn(decay, w));
+}
+
 // Device-side error bits (also the bits of the per-matrix status words).
 constexpr int kStatusNonFinite = 1;
 constexpr int kStatusTimeout = 2;

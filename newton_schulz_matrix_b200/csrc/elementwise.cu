@@ -247,7 +247,7 @@ unpack_kernel(const UnpackArgs a, const __grid_constant__ SegmentPtrs p) {
   if (full) {
     if (UPDATE) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) w[i] = a.decay * w[i] - a.step * o[i];
+      for (int i = 0; i < 16; ++i) w[i] = weight_update(w[i], o[i], a.decay, a.step);
     } else {
 #pragma unroll
       for (int i = 0; i < 16; ++i) w[i] = o[i];
@@ -259,7 +259,7 @@ unpack_kernel(const UnpackArgs a, const __grid_constant__ SegmentPtrs p) {
       const int c = c0 + lc + i;
       if (c < a.cols) {
         const long long o2 = (long long)r * a.cols + c;
-        float v = UPDATE ? a.decay * to_f32(dst[o2]) - a.step * o[i] : o[i];
+        float v = UPDATE ? weight_update(to_f32(dst[o2]), o[i], a.decay, a.step) : o[i];
         dst[o2] = from_f32<TD>(v);
       }
     }
@@ -354,6 +354,17 @@ void launch_unpack(const UnpackArgs& a, const SegmentPtrs& p, cudaStream_t s) {
     case kFP16: unpack_dispatch1<__half>(a, p, s); break;
     default: unpack_dispatch1<float>(a, p, s); break;
   }
+}
+
+__global__ void status_or_kernel(int* status, int count, const int* chunk_err) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int e = *chunk_err;
+  if (i < count && e != 0) status[i] |= e;
+}
+
+void launch_status_or(int* status, int count, const int* chunk_err, cudaStream_t s) {
+  if (count <= 0 || status == nullptr) return;
+  status_or_kernel<<<(count + 255) / 256, 256, 0, s>>>(status, count, chunk_err);
 }
 
 void launch_convert(const void* src, int sdt, void* dst, int ddt, long long n, cudaStream_t s) {

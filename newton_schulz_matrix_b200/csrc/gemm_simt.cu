@@ -305,7 +305,8 @@ ns_fused_small_kernel(const FusedSmallArgs a) {
       smem_mm<false>(Q, ldn, Qa, ldn, Qb, ldn, n, n, n, 1.f, nullptr, 0, 0.f, 0.f, red);      // Q_acc <- Q Q_acc
       float* t = Qa; Qa = Qb; Qb = t;
       if (k == a.iters) break;
-      if (a.restart_after > 0 && k == a.restart_after) {
+      if (a.restart_after > 0 && k >= a.restart_after &&
+          (k == a.restart_after || (a.restart_every > 0 && (k - a.restart_after) % a.restart_every == 0))) {
         smem_mm<false>(Qa, ldn, X, ldx, Y, ldx, n, m, n, 1.f, nullptr, 0, 0.f, 0.f, red);     // X <- Q_acc X0
         float* u = X; X = Y; Y = u;
         smem_mm<true>(X, ldx, X, ldx, R, ldn, n, n, m, 1.f, nullptr, 0, 0.f, 0.f, red);       // R <- X X^T

@@ -26,6 +26,7 @@
 // raises the timeout bit in the caller's error word and returns.
 #include <stdio.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include <atomic>
 
@@ -278,6 +279,41 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMa
 
 }  // namespace tc
 
+namespace {
+// 256-row products go to the paired-CTA kernel (a third less operand
+// traffic per MMA); MUON_GEMM_PAIR=0 keeps every product on the 1-CTA one.
+bool use_pair_kernel(const GemmDesc& g) {
+  static const int use_pair = [] {
+    const char* e = getenv("MUON_GEMM_PAIR");
+    return (e && e[0] == '0') ? 0 : 1;
+  }();
+  return use_pair && g.M >= 256;
+}
+}  // namespace
+
+bool gemm_tc_paired(int M) {
+  GemmDesc g{};
+  g.M = M;
+  return use_pair_kernel(g);
+}
+
+double gemm_tc_exec_flops(const GemmDesc& g) {
+  using namespace tc;
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return 0.0;
+  const double k_pad = (double)((g.K + BK - 1) / BK) * BK;
+  double per_batch = 0.0;  // sum over launched tiles of tile_rows * tile_cols
+  if (use_pair_kernel(g)) {
+    const int tm = (g.M + 255) / 256, tn = (g.N + 255) / 256;
+    const bool narrow = g.N - (tn - 1) * 256 <= 128;  // last column tile runs N = 128 MMAs
+    for (int r = 0; r < tm; ++r)
+      for (int c = g.symmetric ? r : 0; c < tn; ++c) per_batch += 256.0 * ((c == tn - 1 && narrow) ? 128 : 256);
+  } else {
+    const int tm = (g.M + BM - 1) / BM, tn = (g.N + BN - 1) / BN;
+    for (int r = 0; r < tm; ++r) per_batch += (double)(tn - (g.symmetric ? r / 2 : 0)) * BM * BN;
+  }
+  return 2.0 * per_batch * k_pad * g.batch;
+}
+
 int gemm_tc(const GemmDesc& g, cudaStream_t s) {
   using namespace tc;
   if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return 0;
@@ -305,14 +341,11 @@ int gemm_tc(const GemmDesc& g, cudaStream_t s) {
   p.scale = g.scale; p.scale_pow = g.scale_pow;
   p.err = g.err;
   p.timeout_ns = wait_timeout_ns();
+  p.tile_counter = g.tile_counter;
+  p.static_order = static_tile_order() ? 1 : 0;
 
-  // 256-row products go to the paired-CTA kernel (a third less operand
-  // traffic per MMA); MUON_GEMM_PAIR=0 keeps every product on the 1-CTA one.
-  static const int use_pair = [] {
-    const char* e = getenv("MUON_GEMM_PAIR");
-    return (e && e[0] == '0') ? 0 : 1;
-  }();
-  if (use_pair && g.M >= 256) return gemm_tc_pair(g, p, s);
+  if (use_pair_kernel(g)) return gemm_tc_pair(g, p, s);
+  if (g.update != nullptr) return (int)cudaErrorInvalidValue;  // the fused update is a paired-kernel epilogue
 
   CUtensorMap ma, mb;
   if (!encode_map(&ma, g.in_dtype, g.A, g.K, g.M, g.batch, g.lda, g.a_bs, BK, BM)) return (int)cudaErrorInvalidValue;
@@ -331,6 +364,14 @@ int gemm_tc(const GemmDesc& g, cudaStream_t s) {
   }
   if (bmn) return fmt ? launch<true, 1, false>(ma, mb, md, p, s) : launch<true, 0, false>(ma, mb, md, p, s);
   return fmt ? launch<false, 1, false>(ma, mb, md, p, s) : launch<false, 0, false>(ma, mb, md, p, s);
+}
+
+bool tc::static_tile_order() {
+  static const bool on = [] {
+    const char* e = getenv("MUON_TILE_ORDER");
+    return e && strcmp(e, "static") == 0;
+  }();
+  return on;
 }
 
 int current_device() {

@@ -14,11 +14,21 @@
 //     the leader's MMA issuer through a remote mbarrier arrive;
 //   - a ragged last column tile with at most 128 valid columns (e.g. 1408 =
 //     5.5 x 256) runs N = 128 MMAs, each CTA supplying 64 columns, which halves
-//     its tensor work; its accumulator's upper 128 columns are never stored.
+//     its tensor work; its accumulator's upper 128 columns are never stored;
+//   - tiles are handed out dynamically: the leader's producer takes the next
+//     tile index from a device counter (one atomic per tile) and publishes it
+//     in a small ring in both CTAs' shared memory, which the MMA issuer, the
+//     peer's producer and every epilogue warp follow.  All pairs therefore
+//     work on a window of consecutive tiles at any time, so tiles that share an
+//     operand panel run together and read it from L2.  (A fixed round-robin
+//     assignment lets pairs drift apart over a long launch, and with 341
+//     matrices per launch that tripled the DRAM reads of the products.)
 // Waits are bounded as in the 1-CTA kernel.
 #include <stdio.h>
+#include <stdlib.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "tc_common.cuh"
 
@@ -30,7 +40,13 @@ constexpr int STAGES2 = 6;
 constexpr int A_BYTES2 = BM * BK * 2;   // this CTA's 128 rows of A: 16 KB
 constexpr int B_BYTES2 = 128 * BK * 2;  // this CTA's 128 columns of B: 16 KB
 constexpr int STAGE_BYTES2 = A_BYTES2 + B_BYTES2;
-constexpr int SMEM_BYTES2 = STAGES2 * STAGE_BYTES2 + STAGING_BYTES + 1024 + 256;
+constexpr int RING = 8;                 // tile indices in flight from the scheduler to the roles following it
+// arrivals that free a ring slot: the MMA issuer, the peer's producer, and
+// the epilogue warps of both CTAs
+constexpr int RING_CONSUMERS = 1 + 1 + 2 * NUM_EPI_WARPS;
+constexpr int BAR_BYTES2 = 512;         // barriers, the ring, the TMEM address, the abort flag
+constexpr int SMEM_BYTES2 = STAGES2 * STAGE_BYTES2 + STAGING_BYTES + 1024 + BAR_BYTES2;
+static_assert((2 * STAGES2 + 5 + 2 * RING) * 8 + RING * 4 + 8 <= BAR_BYTES2, "barrier area");
 
 __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y, int z) {
@@ -49,11 +65,18 @@ __device__ __forceinline__ void mma_pair(uint32_t d_tmem, uint64_t adesc, uint64
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-template <bool B_MN, int IN_FMT, bool SYM>
+// Kernel parameter of launches without the fused update (keeps their
+// parameter block small; UpdateSlots is ~7 KB).
+struct NoUpdate {
+  int unused;
+};
+
+template <bool B_MN, int IN_FMT, bool SYM, bool UPD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
-            const __grid_constant__ CUtensorMap tmap_d,
-                 const __grid_constant__ Params p) {
+                 const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ Params p,
+                 const __grid_constant__ std::conditional_t<UPD, UpdateSlots, NoUpdate> u) {
+  static_assert(!(UPD && SYM), "the fused update follows a non-symmetric product");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + STAGES2 * STAGE_BYTES2;  // per epilogue warp: two 1024-aligned 2 KB boxes
@@ -63,13 +86,15 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   uint64_t* tfull_bar = bars + 2 * STAGES2;       // [2]         (both CTAs)
   uint64_t* tempty_bar = bars + 2 * STAGES2 + 2;  // [2]         (used in the leader)
   uint64_t* drain_bar = bars + 2 * STAGES2 + 4;   // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES2 + 5);
+  uint64_t* ring_full = bars + 2 * STAGES2 + 5;   // [RING]      (both CTAs)
+  uint64_t* ring_empty = ring_full + RING;        // [RING]      (used in the leader)
+  int* tile_ring = reinterpret_cast<int*>(ring_empty + RING);  // [RING] (both CTAs)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_ring + RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();  // 0 = leader, 1 = peer
   const bool leader = rank == 0;
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES2; ++s) {
@@ -81,6 +106,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       mbar_init(smem_u32(&tempty_bar[a]), 2 * NUM_EPI_WARPS);
     }
     mbar_init(smem_u32(drain_bar), 1);
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(smem_u32(&ring_full[r]), 1);
+      mbar_init(smem_u32(&ring_empty[r]), RING_CONSUMERS);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -100,10 +129,30 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
+  // Programmatic dependent launch: the set-up above may overlap the previous
+  // kernel's last tiles; nothing below reads global memory before that kernel
+  // has finished and its writes are visible.  The next kernel may be scheduled
+  // now (its CTAs need a whole SM's shared memory, so they start on the SMs
+  // this grid leaves).  Both are no-ops when the launch does not use it.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = (p.K + BK - 1) / BK;
   const uint32_t leader_full = mapa(smem_u32(full_bar), 0);
   const uint32_t leader_tempty = mapa(smem_u32(tempty_bar), 0);
+  const uint32_t leader_ring_empty = mapa(smem_u32(ring_empty), 0);
+  // Tile index number i of this pair (in order; -1 once the launch's tiles are
+  // exhausted).  The leader's producer takes it from the counter and
+  // publishes it in both CTAs; every other role reads it from its own CTA's
+  // ring and frees the slot in the leader.  false on timeout or abort.
+  auto next_tile = [&](int i, int& t) -> bool {
+    const int slot = i % RING;
+    const uint32_t rph = (uint32_t)(i / RING) & 1u;
+    if (!mbar_wait_cluster(smem_u32(&ring_full[slot]), rph, abort_flag, p.timeout_ns)) return false;
+    t = tile_ring[slot];
+    remote_arrive(leader_ring_empty + slot * 8);
+    return true;
+  };
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producers (both CTAs)
@@ -111,7 +160,33 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = pair; t < p.total_tiles && ok; t += npairs) {
+      // the scheduler (leader) takes tile indices one ahead: the next index is
+      // requested while this tile's loads go out, so the atomic's latency stays
+      // off the pipeline; MUON_TILE_ORDER=static hands them out round-robin
+      const int pair = (int)(blockIdx.x >> 1), npairs = (int)(gridDim.x >> 1);
+      auto take = [&](int i) -> int {
+        const int t = p.static_order ? pair + i * npairs : atomicAdd(p.tile_counter, 1);
+        return t < p.total_tiles ? t : -1;
+      };
+      int held = leader ? take(0) : -1;
+      for (int i = 0; ok; ++i) {
+        int t;
+        if (leader) {
+          // scheduler: wait until every role has taken index i - RING from this slot
+          const int slot = i % RING;
+          if (!mbar_wait_cluster(smem_u32(&ring_empty[slot]), ((uint32_t)(i / RING) & 1u) ^ 1u, abort_flag,
+                                 p.timeout_ns))
+            break;
+          t = held;
+          if (t >= 0) held = take(i + 1);
+          tile_ring[slot] = t;
+          st_cluster_s32(mapa(smem_u32(&tile_ring[slot]), 1), t);
+          remote_arrive(mapa(smem_u32(&ring_full[slot]), 0));
+          remote_arrive(mapa(smem_u32(&ring_full[slot]), 1));
+        } else if (!next_tile(i, t)) {
+          break;
+        }
+        if (t < 0) break;
         const PairTile tl = decode_pair(p, t);
         // a ragged last column tile with at most 128 valid columns runs N = 128
         // MMAs: each CTA then supplies 64 columns (the first 64 it loads)
@@ -146,7 +221,9 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int t = pair; t < p.total_tiles && ok; t += npairs, ++it) {
+      for (int i = 0; ok; ++i, ++it) {
+        int t;
+        if (!next_tile(i, t) || t < 0) break;
         const uint32_t idesc = p.N - decode_pair(p, t).TN * 256 <= 128 ? idesc_narrow : idesc_full;
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
@@ -182,7 +259,12 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
     uint8_t* S = staging + (warp - 2) * 2 * STAGE_TILE_BYTES;
     uint8_t* T = S + STAGE_TILE_BYTES;
     int it = 0;
-    for (int t = pair; t < p.total_tiles; t += npairs, ++it) {
+    for (int ti = 0;; ++ti, ++it) {
+      int t = -1, got = 1;
+      if (lane == 0) got = next_tile(ti, t);
+      got = __shfl_sync(0xffffffffu, got, 0);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (!got || t < 0) break;
       const PairTile pt = decode_pair(p, t);
       const Tile tl{pt.b, pt.TM * 2 + (int)rank, pt.TN};
       const int acc = it & 1;
@@ -215,7 +297,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           __syncwarp();
           if (lane == 0) remote_arrive(leader_tempty + acc * 8);
         }
-        epilogue_chunk<SYM>(p, &tmap_d, tl, q, lane, c, r, creg, c_ready, f, S, T);
+        if constexpr (UPD) {
+          update_chunk(p, u, tl, q, lane, c, r, creg, c_ready, f, S);
+        } else {
+          epilogue_chunk<SYM>(p, &tmap_d, tl, q, lane, c, r, creg, c_ready, f, S, T);
+        }
       }
     }
     if (lane == 0) bulk_wait_all0();  // this warp's output stores have completed
@@ -233,20 +319,32 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   if (threadIdx.x == 0 && *abort_flag && p.err != nullptr) atomicOr(p.err, kStatusTimeout);
 }
 
-template <bool B_MN, int IN_FMT, bool SYM>
+// Product launches may start while the previous kernel on the stream drains
+// (programmatic dependent launch); MUON_PDL=0 launches them fully serialised.
+static bool programmatic_launch() {
+  static const bool on = [] {
+    const char* e = getenv("MUON_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+template <bool B_MN, int IN_FMT, bool SYM, bool UPD = false, typename Slots = NoUpdate>
 static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
-                  cudaStream_t s) {
+                  cudaStream_t s, const Slots& u = Slots{}) {
   // per device: shared-memory opt-in done and how many CTA pairs fit at once
   static std::atomic<int> max_pairs_of[kMaxDevices];
   const int dev = current_device();
   if (dev < 0) return (int)cudaErrorInvalidDevice;
-  auto kern = gemm_pair_kernel<B_MN, IN_FMT, SYM>;
+  auto kern = gemm_pair_kernel<B_MN, IN_FMT, SYM, UPD>;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = SMEM_BYTES2;
   cfg.stream = s;
@@ -265,7 +363,8 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMa
   }
   const int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   cfg.gridDim = dim3(2 * pairs);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p);
+  cfg.numAttrs = programmatic_launch() ? 2 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p, u);
   return (int)e;
 }
 
@@ -273,6 +372,7 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMa
 
 int gemm_tc_pair(const GemmDesc& g, Params p, cudaStream_t s) {
   using namespace pairk;
+  if (p.tile_counter == nullptr) return (int)cudaErrorInvalidValue;
   // pair tiles: 256 rows x 256 columns
   p.tiles_m = (g.M + 255) / 256;
   p.tiles_n = (g.N + BN - 1) / BN;
@@ -295,6 +395,12 @@ int gemm_tc_pair(const GemmDesc& g, Params p, cudaStream_t s) {
   CUtensorMap md;
   if (!encode_out_map(&md, g)) return (int)cudaErrorInvalidValue;
   const int fmt = g.in_dtype == kBF16 ? 1 : 0;
+  if (g.update != nullptr) {
+    // the fused update follows the chain's last product: X' = a X + B X (B MN-major)
+    if (g.symmetric || !bmn || g.batch > UpdateSlots::kMax) return (int)cudaErrorInvalidValue;
+    return fmt ? launch<true, 1, false, true>(ma, mb, md, p, s, *g.update)
+               : launch<true, 0, false, true>(ma, mb, md, p, s, *g.update);
+  }
   if (g.symmetric) {
     if (bmn) return fmt ? launch<true, 1, true>(ma, mb, md, p, s) : launch<true, 0, true>(ma, mb, md, p, s);
     return fmt ? launch<false, 1, true>(ma, mb, md, p, s) : launch<false, 0, true>(ma, mb, md, p, s);

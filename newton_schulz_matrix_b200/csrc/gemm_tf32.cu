@@ -475,6 +475,16 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMa
 }  // namespace tf32k
 }  // namespace tc
 
+double gemm_tf32x3_exec_flops(const GemmDesc& g) {
+  using namespace tc::tf32k;
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return 0.0;
+  const int tm = (g.M + 255) / 256, tn = (g.N + TILE_N - 1) / TILE_N;
+  double tiles = 0.0;
+  for (int r = 0; r < tm; ++r) tiles += g.symmetric ? tn - 2 * r : tn;
+  const double k_pad = (double)((g.K + BK32 - 1) / BK32) * BK32;
+  return 3.0 * 2.0 * tiles * 256.0 * TILE_N * k_pad * g.batch;  // hi*hi + hi*lo + lo*hi
+}
+
 int gemm_tf32x3(const GemmDesc& g, cudaStream_t s) {
   using namespace tc;
   using namespace tc::tf32k;

@@ -60,7 +60,24 @@ void launch_unpack(const UnpackArgs& a, const SegmentPtrs& p, cudaStream_t s);
 void launch_convert(const void* src, int src_dtype, void* dst, int dst_dtype, long long n,
                     cudaStream_t s);
 
+// status[i] |= *chunk_err for i < count (the chunk's device-side error bits,
+// e.g. a wait timeout, reported to every matrix of the chunk).
+void launch_status_or(int* status, int count, const int* chunk_err, cudaStream_t s);
+
 // ---------------------------------------------------------------- products
+// The last product of a Muon step's chain can write the update itself: its
+// epilogue rounds O to the chain's type (as the stored X would be) and writes
+// W <- decay W - step O for every matrix of the launch, in W's storage
+// orientation, instead of storing O (the paired-CTA kernel; see run_batches).
+struct UpdateSlots {
+  static constexpr int kMax = 512;  // matrices per launch (kernel-parameter space)
+  float decay, step;                // decay = 1 - lr wd, step = lr scale_coef sqrt(max(r, c))
+  int* status;                      // per-matrix status words (may be null)
+  void* w[kMax];                    // W of batch index b
+  int status_idx[kMax];             // its index into status
+  unsigned char kind[kMax];         // bit 0: stored transposed (m x n); bits 1-2: W dtype
+};
+
 // D[b] = epilogue(A[b] * op(B[b])) for b < batch, all row-major.
 //   A is M x K (K contiguous).  op(B) is K x N given either as rows of
 //   length K (b_kmajor = 1: B stored N x K, i.e. D = A B^T) or as rows of
@@ -79,9 +96,26 @@ struct GemmDesc {
   const float* scale; int scale_pow;
   int symmetric;
   int* err;               // device word: timeout bits land here (may be null)
+  int* tile_counter;      // device word, 0 before the launch: the paired-CTA kernel's tile scheduler
+  const UpdateSlots* update;  // host struct: write the Muon update instead of D (non-symmetric, M >= 256)
 };
 // Tensor-core (tcgen05) path: bf16/fp16 operands.  Returns 0 or a CUDA error.
 int gemm_tc(const GemmDesc& g, cudaStream_t s);
+// Whether gemm_tc runs an M-row product on the paired-CTA kernel (the one
+// that can write the fused update).
+bool gemm_tc_paired(int M);
+// A chain of n <= 24 products (16-bit, M >= 256, one batch size, one operand
+// type) as one persistent launch; product i waits, per matrix, for product
+// i - 1 (see gemm_chain.cu).  tile_counter: one zeroed word; done: n * batch
+// zeroed words.  Only the last product may carry `update`.
+int gemm_chain(const GemmDesc* prods, int n, int* tile_counter, int* done, int* err, cudaStream_t s);
+constexpr int kChainMaxProducts = 24;
+// FLOPs the tensor cores execute for one gemm_tc / gemm_tf32x3 launch of `g`:
+// every MMA over whole tiles (zero padding of ragged tiles and k-blocks
+// included), only the tiles a symmetric product computes, and for 3xTF32 the
+// three MMAs per product term.  The algorithmic count is 2 M N K per matrix.
+double gemm_tc_exec_flops(const GemmDesc& g);
+double gemm_tf32x3_exec_flops(const GemmDesc& g);
 // Tensor-core path for fp32 operands (3xTF32, paired CTAs): fp32 A, B, C and D.
 int gemm_tf32x3(const GemmDesc& g, cudaStream_t s);
 // SIMT path (any dtype, fp32 math): fp32 products with fewer than 256 rows.
@@ -97,6 +131,7 @@ struct FusedSmallArgs {
   const float* inv; int raw;
   int mode;            // 0 standard, 1 Gram (restart_after 0 = naive)
   int restart_after;
+  int restart_every;   // 0: restart once; e > 0: also every e iterations after it
   int iters;
   float coeffs[3 * kMaxIters];
 };

@@ -38,6 +38,8 @@ struct Params {
   const float* scale; int scale_pow;
   int* err;
   long long timeout_ns;
+  int* tile_counter;      // paired-CTA kernel: device word, 0 at launch; tiles are taken from it in order
+  int static_order;       // 1: tiles round-robin over the pairs instead (comparison runs)
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -324,6 +326,136 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMa
   }
 }
 
+// ------------------------------------------------------------------ fused Muon update
+// Load / update / store 16 consecutive W elements at `w` (16-byte aligned when
+// `vec`; otherwise only the first `valid` are touched, one by one).
+__device__ __forceinline__ void update16(char* w, int wdt, const float* o, int valid, bool vec, float decay,
+                                         float step) {
+  if (vec) {
+    if (wdt == kFP32) {
+      float4* q = reinterpret_cast<float4*>(w);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float4 x = q[k];
+        x.x = weight_update(x.x, o[4 * k], decay, step);
+        x.y = weight_update(x.y, o[4 * k + 1], decay, step);
+        x.z = weight_update(x.z, o[4 * k + 2], decay, step);
+        x.w = weight_update(x.w, o[4 * k + 3], decay, step);
+        q[k] = x;
+      }
+    } else {
+      uint4* q = reinterpret_cast<uint4*>(w);
+      uint4 x[2] = {q[0], q[1]};
+      float v[16];
+      if (wdt == kBF16) {
+        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(x);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = weight_update(__bfloat162float(e[k]), o[k], decay, step);
+        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(x);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) d[k] = __float2bfloat16_rn(v[k]);
+      } else {
+        const __half* e = reinterpret_cast<const __half*>(x);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = weight_update(__half2float(e[k]), o[k], decay, step);
+        __half* d = reinterpret_cast<__half*>(x);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) d[k] = __float2half_rn(v[k]);
+      }
+      q[0] = x[0];
+      q[1] = x[1];
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (k < valid) store_any(w, k, wdt, weight_update(load_any(w, k, wdt), o[k], decay, step));
+  }
+}
+
+// The fused-update counterpart of epilogue_chunk (non-symmetric products):
+// O = f (c_acc acc + c_in C) for this warp's 32 rows x 32 columns, rounded to
+// the chain's type as the stored X would be, then W <- decay W - step O for
+// matrix t.b.  A matrix stored transposed (m x n) goes through this warp's
+// staging box, so that each lane then updates one contiguous W row segment.
+// Non-finite O raises MUON_STATUS_NONFINITE in the matrix's status word.
+template <typename Slots>
+__device__ __forceinline__ void update_chunk(const Params& p, const Slots& u, const Tile& t, int q, int lane,
+                                             int chunk, const uint32_t (&acc)[32], const uint4 (&creg)[4],
+                                             bool c_ready, float f, uint8_t* S) {
+  const int gi_base = t.tm * BM + q * 32;
+  const int gi = gi_base + lane;
+  const int gj0 = t.tn * BN + chunk * 32;
+  if (gj0 >= p.N || gi_base >= p.M) return;  // warp-uniform
+  float v[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = p.c_acc * __uint_as_float(acc[j]);
+  if (p.C != nullptr && gi < p.M) {
+    if (c_ready) {
+      float c[32];
+      cvt_row32(creg, p.c_dtype, c);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] += p.c_in * c[j];
+    } else {
+      const char* cb = reinterpret_cast<const char*>(p.C) + (long long)t.b * p.c_bs * 2;
+      const long long off = (long long)gi * p.ldc + gj0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (gj0 + j < p.N) v[j] += p.c_in * load_any(cb, off + j, p.c_dtype);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    v[j] *= f;
+    if (gj0 + j == gi) v[j] += p.c_eye;
+  }
+  uint4 oq[4];
+  pack_row32(v, p.d_dtype, oq);   // O in the chain's storage type
+  cvt_row32(oq, p.d_dtype, v);
+  int bad = 0;
+  if (gi < p.M) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) bad |= (gj0 + j < p.N) && !isfinite(v[j]);
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad && lane == 0 && u.status != nullptr) atomicOr(u.status + u.status_idx[t.b], kStatusNonFinite);
+
+  const unsigned kind = u.kind[t.b];
+  const int wdt = (int)(kind >> 1);
+  const int es = wdt == kFP32 ? 4 : 2;
+  char* W = reinterpret_cast<char*>(u.w[t.b]);
+  if (!(kind & 1u)) {
+    // W is M x N like O: this lane's row gi, columns gj0 .. gj0 + 31
+    if (gi < p.M) {
+      char* row = W + ((long long)gi * p.N + gj0) * es;
+      const int valid = min(32, p.N - gj0);
+      const bool vec = valid == 32 && ((long long)p.N * es) % 16 == 0;
+      update16(row, wdt, v, min(16, valid), vec, u.decay, u.step);
+      if (valid > 16) update16(row + 16 * es, wdt, v + 16, valid - 16, vec, u.decay, u.step);
+    }
+  } else {
+    // W is N x M: transpose the 32 x 32 box of O through shared memory, then
+    // lane L updates W row gj0 + L, columns gi_base .. gi_base + 31
+    const uint16_t* ob = reinterpret_cast<const uint16_t*>(oq);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      *reinterpret_cast<uint16_t*>(S + sw64(j, lane >> 3) + (lane & 7) * 2) = ob[j];
+    __syncwarp();
+    uint4 tq[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) tq[k] = *reinterpret_cast<const uint4*>(S + sw64(lane, k));
+    float o[32];
+    cvt_row32(tq, p.d_dtype, o);
+    if (gj0 + lane < p.N) {
+      char* row = W + ((long long)(gj0 + lane) * p.M + gi_base) * es;
+      const int valid = min(32, p.M - gi_base);
+      const bool vec = valid == 32 && ((long long)p.M * es) % 16 == 0;
+      update16(row, wdt, o, min(16, valid), vec, u.decay, u.step);
+      if (valid > 16) update16(row + 16 * es, wdt, o + 16, valid - 16, vec, u.decay, u.step);
+    }
+  }
+}
+
 // ------------------------------------------------------------------ clusters of two CTAs
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -349,6 +481,41 @@ __device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t mask) {
 }
 __device__ __forceinline__ void remote_arrive(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// Store to the same shared-memory object in another CTA of the cluster (address from mapa).
+__device__ __forceinline__ void st_cluster_s32(uint32_t addr_cluster, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
+}
+// Wait on a barrier of this CTA whose arrivals (and the data they publish)
+// come from other CTAs of the cluster: acquire at cluster scope.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded as mbar_wait: false when the deadline passed or another role aborted.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  long long timeout_ns) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer();
+  for (uint32_t it = 1; it < (1u << 30); ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 31u) == 0) {
+      if (*abort_flag) return false;
+      if ((long long)(global_timer() - t0) > timeout_ns) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+  *abort_flag = 1;
+  return false;
 }
 
 // Tile order of the paired-CTA kernels: 256 x 256 tiles (upper triangle only
@@ -379,6 +546,33 @@ __device__ __forceinline__ PairTile decode_pair(const Params& p, int t) {
   }
   return r;
 }
+
+// ------------------------------------------------------------------ whole chains in one launch (gemm_chain.cu)
+// One product of a chain launch: its operand and output maps, shape, tile
+// range in the launch's tile space, epilogue and the product it depends on.
+struct alignas(64) ChainProduct {
+  CUtensorMap ma, mb, md;
+  int M, N, K, batch;
+  int tiles_m, tiles_n, tiles_per_batch, first_tile;
+  int symmetric, b_mn, dep;
+  void* D; int ldd; long long d_bs; int d_dtype;
+  const void* C; int ldc; long long c_bs; int c_dtype;
+  float c_acc, c_in, c_eye;
+  const float* scale; int scale_pow;
+};
+struct ChainParams {
+  static constexpr int kMaxProducts = 24;
+  int n_products, batch, total_tiles, static_order;
+  int* tile_counter;      // device word, 0 at launch
+  int* done;              // [n_products][batch] arrival counters, 0 at launch
+  int* err;
+  long long timeout_ns;
+  ChainProduct prod[kMaxProducts];
+};
+
+// Tiles from the counter (default) or round-robin (MUON_TILE_ORDER=static):
+// the same tiles and arithmetic either way, only the hand-out order differs.
+bool static_tile_order();
 
 // ------------------------------------------------------------------ host side (gemm_tc.cu)
 // 3-D tiled tensor map over a batch of row-major matrices.  Shared-memory

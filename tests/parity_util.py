@@ -1,16 +1,18 @@
 """Shared helpers of the GPU parity tests: oracle calls, tolerances, sigma band.
 
-Tolerance rule (derived from the arithmetic; the numbers behind it are in the
-design notes): fp32 compute must match the fp64 oracle within 1e-4 relative
-Frobenius error.  bf16/fp16 compute must match within 2e-2, or within 1.25 x the
-error that the oracle's own storage-rounding emulation shows on the same input
-when that floor is above 1.6e-2 (ill-conditioned spectra, where any 16-bit
-execution mixes singular vectors of nearly equal singular values); and in both
-cases every output singular value must lie within 0.05 of the value the
-iteration maps the matching input singular value to (the sigma band).
-"""
-from __future__ import annotations
+Tolerances: fp32 compute must match the fp64 oracle within 1e-4 relative
+Frobenius error, 16-bit compute within 2e-2, and every output singular value
+must lie within 0.05 of the value the iteration maps the matching input
+singular value to (the sigma band).
 
+One exception, used only where a test says so: on ill-conditioned spectra no
+16-bit execution of some forms can reach 2e-2 (bf16 storage of the standard
+form; the naive fp16 Gram form, which the write-up calls unstable).  There the
+bound is 1.25 x the error of the oracle's stored-precision iteration on the
+same input (``oracle.ns_standard_stored`` / ``ns_gram_stored``, pinned in
+test_oracle_pins.py), i.e. the GPU may add at most a quarter of what the
+storage type's own rounding already costs.
+"""
 import math
 
 import numpy as np
@@ -34,32 +36,41 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def emulated_output(U: np.ndarray, coeffs, mode: str, restart_after=2, gram_fmt="fp16", x_fmt="bf16"):
-    """(exact, emulated) oriented outputs: the iteration in fp64 and with every
-    stored matrix rounded to its 16-bit storage type (oracle emulation)."""
+def emulated_output(U: np.ndarray, coeffs, mode: str, restart_after=2, chain="fp16", eps=1e-7):
+    """(exact, stored) oriented outputs for the input U: the fp64 iteration, and
+    the iteration with every product stored in ``chain`` (the chain's 16-bit
+    type: compute_dtype for the standard form, gram_dtype for the Gram forms).
+    As in the kernels, a bf16 chain starts from the raw U rounded to bf16 and
+    applies f = 1 / (||U||_F + eps) inside the first products, and an fp16 chain
+    starts from X0 = f U rounded once to fp16."""
     X, _ = oracle.orient(U)
-    X0 = oracle.frobenius_normalize(X)
-    exact = oracle.ns_standard(X0, coeffs)
-    if mode == "standard":
-        emu = oracle.ns_standard(oracle.round_to(X0, x_fmt), coeffs, emulate=x_fmt)
+    f = 1.0 / (oracle.frobenius_norm(X) + eps)
+    exact_in = X * f
+    exact = oracle.ns_standard(exact_in, coeffs) if mode == "standard" else oracle.ns_gram(
+        exact_in, coeffs, 0 if mode == "gram" else restart_after)
+    if chain == "bf16":
+        start, prescale = oracle.round_to(X, "bf16"), f
     else:
-        x_fmt = gram_fmt  # the Gram chain stores X0 and the restart X in the Gram type too
+        start, prescale = oracle.round_to(exact_in, chain), None
+    if mode == "standard":
+        emu = oracle.ns_standard_stored(start, coeffs, chain, prescale=prescale)
+    else:
         ra = 0 if mode == "gram" else restart_after
-        emu = oracle.ns_gram(oracle.round_to(X0, x_fmt), coeffs, ra, emulate_gram=gram_fmt, emulate_x=x_fmt)
+        emu = oracle.ns_gram_stored(start, coeffs, chain, ra, prescale=prescale)
     return exact, emu
 
 
-def emulated_floor(U: np.ndarray, coeffs, mode: str, restart_after=2, gram_fmt="fp16", x_fmt="bf16") -> float:
-    """Relative error of a 16-bit-storage execution of the iteration (oracle emulation)."""
-    exact, emu = emulated_output(U, coeffs, mode, restart_after, gram_fmt, x_fmt)
+def emulated_floor(U: np.ndarray, coeffs, mode: str, restart_after=2, chain="fp16") -> float:
+    """Relative error of a 16-bit-storage execution of the iteration on U."""
+    exact, emu = emulated_output(U, coeffs, mode, restart_after, chain)
     return rel(emu, exact) if np.all(np.isfinite(emu)) else math.inf
 
 
-def emulated_band_holds(U: np.ndarray, coeffs, mode: str, restart_after=2, gram_fmt="fp16") -> bool:
+def emulated_band_holds(U: np.ndarray, coeffs, mode: str, restart_after=2, chain="fp16") -> bool:
     """Whether the 16-bit execution itself keeps the sigma band on this input
     (the naive Gram form does not on ill-conditioned spectra: the write-up's
     float16 instability)."""
-    _, emu = emulated_output(U, coeffs, mode, restart_after, gram_fmt)
+    _, emu = emulated_output(U, coeffs, mode, restart_after, chain)
     if not np.all(np.isfinite(emu)):
         return False
     Xo, tr = oracle.orient(U)
@@ -67,11 +78,18 @@ def emulated_band_holds(U: np.ndarray, coeffs, mode: str, restart_after=2, gram_
 
 
 def tolerance(compute: str, floor: float | None = None) -> float:
+    """The stated bar for ``compute``; with ``floor`` (only where a test opts
+    into the exception above) max(2e-2, 1.25 x floor)."""
     if compute == "fp32":
         return FP32_TOL
     if floor is None or floor <= BF16_TOL / 1.25:
         return BF16_TOL
     return 1.25 * floor
+
+
+def chain_of(mode: str, compute: str = "fp16", gram_dtype: str = "fp16") -> str:
+    """The storage type of a 16-bit chain (what ``emulated_floor`` takes)."""
+    return compute if mode == "standard" else gram_dtype
 
 
 def sigma_band_error(U: np.ndarray | torch.Tensor, O: np.ndarray | torch.Tensor, coeffs, eps=1e-7) -> float:

@@ -45,8 +45,8 @@ def test_status_strings(lib):
     assert nsm.muon_status_string(99) == "unknown code"
 
 
-def _ns(coeffs=(nsm.QUINTIC,) * 5, mode="standard", restart_after=2, compute="bf16", gram="fp16"):
-    return nsm._ns_params(coeffs, mode, restart_after, 1e-7, compute, gram)
+def _ns(coeffs=(nsm.QUINTIC,) * 5, mode="standard", restart_after=2, compute="bf16", gram="fp16", every=0):
+    return nsm._ns_params(coeffs, mode, restart_after, 1e-7, compute, gram, every)
 
 
 @pytest.mark.parametrize("rows,cols", [(64, 128), (2048, 7168), (7168, 18432), (1408, 2048), (333, 77)])
@@ -55,6 +55,15 @@ def test_flop_counts_agree_with_oracle(lib, rows, cols, mode):
     ns, _a = _ns(mode=mode)
     got = lib.muon_ns_flops(rows, cols, ctypes.byref(ns))
     assert got == float(oracle.flops(rows, cols, 5, mode, 2))
+
+
+@pytest.mark.parametrize("iters,restart,every", [(5, 2, 2), (7, 1, 3), (5, 2, 1), (6, 3, 0)])
+def test_periodic_restart_flop_counts_agree_with_oracle(lib, iters, restart, every):
+    ns, _a = _ns(coeffs=(nsm.QUINTIC,) * iters, mode="gram_stabilized", restart_after=restart, every=every)
+    assert lib.muon_ns_flops(2048, 7168, ctypes.byref(ns)) == float(
+        oracle.flops(2048, 7168, iters, "gram_stabilized", restart, every))
+    bad, _b = _ns(mode="gram_stabilized", every=-1)
+    assert lib.muon_ns_flops(2048, 7168, ctypes.byref(bad)) == 0.0
 
 
 def test_ns_workspace_size(lib):

@@ -13,7 +13,7 @@ import torch
 import newton_schulz_matrix_b200 as nsm
 import oracle
 import synth
-from parity_util import Q5, emulated_band_holds, emulated_floor, rel, sigma_band_error, to_np, tolerance
+from parity_util import Q5, chain_of, emulated_band_holds, emulated_floor, rel, sigma_band_error, to_np, tolerance
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -57,8 +57,14 @@ def run_step(params, grads, moms, ws_bytes=None, **hp):
     return status
 
 
-def check_sample_fp32_w(W0, W1, G, M0, M1, hp, mode):
-    """O recovered exactly from an fp32 W update; checked against the oracle."""
+def check_sample_fp32_w(W0, W1, G, M0, M1, hp, mode, compute="fp16"):
+    """O recovered exactly from an fp32 W update; checked against the oracle.
+
+    The standard form on the default fp16 chain is held to the stated 2e-2.
+    The Gram forms (and any bf16 chain) are held to max(2e-2, 1.25 x the
+    floor of their 16-bit storage on this input): on the dense recipe the fp16
+    Gram chain's own rounding already costs 2.1e-2 (stabilised) and 4.3e-2
+    (naive), on the 1/i spectrum the naive form reaches 0.13."""
     r, c = W0.shape
     Wr, Mr, Or = oracle.muon_step(W0, G, M0, mode=mode, restart_after=2, **hp)
     assert rel(M1, Mr) < 1e-6
@@ -66,9 +72,10 @@ def check_sample_fp32_w(W0, W1, G, M0, M1, hp, mode):
     O = ((1 - hp["lr"] * hp["weight_decay"]) * W0 - W1) / step
     U = oracle.nesterov_blend(G, Mr, hp["momentum"], hp["nesterov"])
     err = rel(O, Or)
-    floor = emulated_floor(U, hp["coeffs"], mode)
-    assert err < tolerance("bf16", floor), (err, floor)
-    if emulated_band_holds(U, hp["coeffs"], mode):
+    strict = mode == "standard" and compute != "bf16"
+    floor = None if strict else emulated_floor(U, hp["coeffs"], mode, chain=chain_of(mode, compute))
+    assert err < tolerance(compute, floor), (err, floor)
+    if emulated_band_holds(U, hp["coeffs"], mode, chain=chain_of(mode, compute)):
         assert sigma_band_error(U, O, hp["coeffs"]) < 0.05
     return err, floor
 
@@ -76,18 +83,19 @@ def check_sample_fp32_w(W0, W1, G, M0, M1, hp, mode):
 # ---------------------------------------------------------------------------
 # 64 x 1024 x 4096 dense projections (rank-64 + noise gradients)
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("mode", ["standard", "gram"])
-def test_dense_projection_batch(mode):
+@pytest.mark.parametrize("mode,compute", [("standard", "fp16"), ("gram", "fp16"), ("gram_stabilized", "fp16"),
+                                          ("standard", "bf16")])
+def test_dense_projection_batch(mode, compute):
     w = synth.dense_projection(device=DEV)
     g = w.groups[0]
     params = [x.float() for x in g.W]   # fp32 W so that O is observable exactly
     W0 = [to_np(p) for p in params[:2]]
     M0 = [to_np(m) for m in g.M[:2]]
     hp = step_hp()
-    status = run_step(params, g.G, g.M, mode=mode, **hp)
+    status = run_step(params, g.G, g.M, mode=mode, compute_dtype=compute, **hp)
     assert int((status != 0).sum()) == 0
     for i in range(2):
-        check_sample_fp32_w(W0[i], to_np(params[i]), to_np(g.G[i]), M0[i], to_np(g.M[i]), hp, mode)
+        check_sample_fp32_w(W0[i], to_np(params[i]), to_np(g.G[i]), M0[i], to_np(g.M[i]), hp, mode, compute)
 
 
 # ---------------------------------------------------------------------------
@@ -142,8 +150,9 @@ def test_kimi_k2_full_step_as_benchmarked():
         q = rel(oracle.round_to(Wr, "bf16") - to_np(W0[i]), dW_ref)
         dW = to_np(params[i]) - to_np(W0[i])
         U = oracle.nesterov_blend(to_np(grads[i]), Mr, hp["momentum"], True)
-        floor = emulated_floor(U, Q5, "standard")
-        assert rel(dW, dW_ref) < tolerance("bf16", math.hypot(floor, q)), (rel(dW, dW_ref), floor, q)
+        # the orthogonalisation is held to the stated 2e-2; the bf16 store of W
+        # adds its own, independent quantisation q of the update on top
+        assert rel(dW, dW_ref) < math.hypot(2e-2, q), (rel(dW, dW_ref), q)
         assert sigma_band_error(U, -(dW - (decay - 1) * to_np(W0[i])) / step, Q5) < 0.05
     # dense matrix: sigma band at full size on the device
     i = dense
@@ -181,12 +190,22 @@ def test_kimi_k2_subset_stabilized_gram():
 
 
 # ---------------------------------------------------------------------------
-# stress sweep: log-uniform spectra in [1e-6, 1], fp16 Gram path
+# stress sweep: log-uniform spectra in [1e-6, 1], all twelve (n, alpha) points
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("n,alpha", [(1024, 1), (1024, 2), (1024, 4), (1024, 8), (2048, 1), (2048, 8)])
+STRESS_POINTS = [(n, a) for n in (1024, 2048, 4096) for a in (1, 2, 4, 8)]
+
+
+@pytest.mark.parametrize("n,alpha", STRESS_POINTS)
 def test_stress_sweep(n, alpha):
+    """Every form on 32 ill-conditioned matrices (default fp16 chains): no
+    Inf/NaN in the standard or stabilised form, the sigma band on the device
+    (fp64 Gram eigenvalues) for matrix 0 at every size, and matrix 0 against
+    the fp64 oracle up to n = 2048 (at n = 4096 the oracle takes minutes per
+    matrix; the same recipe is checked against it at n = 1024 and 2048).  The
+    standard and stabilised forms meet the stated 2e-2; the naive Gram form is
+    held to 1.25 x its own fp16 floor (the write-up's instability)."""
     mats = synth.stress_point(n, alpha, count=32, device=DEV)
-    U0 = to_np(mats[0])
+    U0 = to_np(mats[0]) if n <= 2048 else None
     for mode in ("standard", "gram", "gram_stabilized"):
         ys = [m.clone() for m in mats]
         st = torch.full((32,), -1, dtype=torch.int32, device=DEV)
@@ -195,18 +214,19 @@ def test_stress_sweep(n, alpha):
         flags = st.cpu().numpy()
         if mode != "gram":
             assert int((flags != 0).sum()) == 0  # no Inf/NaN in the standard or stabilised form
-        floor = emulated_floor(U0, Q5, mode)
-        if not math.isfinite(floor):
-            # the fp16 naive Gram form overflows on this spectrum (the write-up's Inf): the
-            # GPU must report it through the status word or stay finite
-            assert flags[0] in (0, 1)
+        if not torch.isfinite(ys[0]).all():
+            # the fp16 naive Gram form may overflow on this spectrum (the write-up's Inf): then
+            # the status word must say so
+            assert mode == "gram" and flags[0] == 1
+            continue
+        assert flags[0] == 0
+        assert sigma_band_gpu(mats[0], ys[0]) < 0.05, mode
+        if U0 is None:
             continue
         want = oracle.newton_schulz(U0, Q5, mode=mode)
-        y0 = to_np(ys[0])
-        assert flags[0] == 0
-        assert rel(y0, want) < tolerance("bf16", floor), (mode, rel(y0, want), floor)
-        if emulated_band_holds(U0, Q5, mode):
-            assert sigma_band_error(U0, y0, Q5) < 0.05
+        floor = emulated_floor(U0, Q5, mode) if mode == "gram" else None
+        assert rel(to_np(ys[0]), want) < tolerance("fp16", floor), (mode, rel(to_np(ys[0]), want), floor)
+        del ys
 
 
 # ---------------------------------------------------------------------------

@@ -11,7 +11,7 @@ import torch
 import newton_schulz_matrix_b200 as nsm
 import oracle
 import synth
-from parity_util import Q5, emulated_band_holds, emulated_floor, rel, sigma_band_error, to_np, tolerance
+from parity_util import Q5, chain_of, emulated_band_holds, emulated_floor, rel, sigma_band_error, to_np, tolerance
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -39,15 +39,24 @@ def gpu_ns(mats, **kw):
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("shape", [(128, 256), (200, 328), (328, 200), (130, 520), (257, 1031)])
 @pytest.mark.parametrize("abc", [(1.0, 0.0, 0.0), (0.0, 1.0, 0.0), (0.0, 0.0, 1.0), (0.5, -0.25, 2.0)])
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_single_iteration_products(shape, abc, dtype):
+@pytest.mark.parametrize("compute", ["bf16", "fp16", "fp32"])
+def test_single_iteration_products(shape, abc, compute):
+    """One product at a time.  The fp16 chain skips the isolated (X X^T)^2 X:
+    on a normalised X it is of order sigma^5 (~1e-5 here), below fp16's normal
+    range, so its relative error measures fp16's subnormal spacing rather than
+    the kernels (in the full iteration the c term is added to a X + b A X and
+    the singular values grow towards 1); the sigma^3 term is partly subnormal
+    too, hence 5e-3 rather than the ~1e-3 of two fp16 roundings."""
+    if compute == "fp16" and abc == (0.0, 0.0, 1.0):
+        pytest.skip("isolated sigma^5 term lies in fp16's subnormal range")
+    dtype = torch.float32 if compute == "fp32" else torch.bfloat16
     X = synth.gaussian(*shape, seed=shape[0] * 7 + 1, device=DEV, dtype=dtype)
-    (Y,), st = gpu_ns([X], coeffs=[abc])
+    (Y,), st = gpu_ns([X], coeffs=[abc], compute_dtype=compute)
     want = oracle.newton_schulz(to_np(X), [abc])
     err = rel(to_np(Y), want)
     assert st == [0]
     # one product: inputs and result each rounded once to the storage type
-    assert err < (1e-5 if dtype == torch.float32 else 8e-3), err
+    assert err < {"fp32": 1e-5, "fp16": 5e-3, "bf16": 8e-3}[compute], err
 
 
 # ---------------------------------------------------------------------------
@@ -55,8 +64,10 @@ def test_single_iteration_products(shape, abc, dtype):
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("mode", ["standard", "gram", "gram_stabilized"])
-@pytest.mark.parametrize("compute", ["bf16", "fp32"])
+@pytest.mark.parametrize("compute", ["fp16", "bf16", "fp32"])
 def test_ns_batched_vs_oracle(shape, mode, compute):
+    """fp32 and the default fp16 chain meet the stated bars outright; the bf16
+    chain is held to its storage type's own floor (at most 1.25 x it)."""
     dtype = torch.float32 if compute == "fp32" else torch.bfloat16
     mats = [synth.gaussian(*shape, seed=100 + i + shape[0], device=DEV, dtype=dtype) for i in range(3)]
     ys, st = gpu_ns(mats, mode=mode, compute_dtype=compute)
@@ -64,7 +75,7 @@ def test_ns_batched_vs_oracle(shape, mode, compute):
     for x, y in zip(mats, ys):
         U = to_np(x)
         want = oracle.newton_schulz(U, Q5, mode=mode)
-        floor = None if compute == "fp32" else emulated_floor(U, Q5, mode)
+        floor = emulated_floor(U, Q5, mode, chain=chain_of(mode, compute)) if compute == "bf16" else None
         err = rel(to_np(y), want)
         assert err < tolerance(compute, floor), (err, floor)
         if min(shape) > 1:
@@ -73,14 +84,16 @@ def test_ns_batched_vs_oracle(shape, mode, compute):
 
 @pytest.mark.parametrize("mode", ["standard", "gram", "gram_stabilized"])
 def test_spectrum_inputs_and_sigma_band(mode):
-    """Power-law spectrum on Haar bases (the MoE recipe), 256 x 1024."""
+    """Power-law spectrum on Haar bases (the MoE recipe), 256 x 1024, default
+    fp16 chain: the stated 2e-2 except for the naive Gram form, which the
+    write-up calls unstable in float16 (held to its own floor)."""
     U = synth.with_spectrum(256, 1024, synth.power_law_sigma(256), 5, device=DEV).bfloat16()
     (y,), st = gpu_ns([U], mode=mode)
     Un = to_np(U)
     want = oracle.newton_schulz(Un, Q5, mode=mode)
-    floor = emulated_floor(Un, Q5, mode)
+    floor = emulated_floor(Un, Q5, mode) if mode == "gram" else None
     assert st == [0]
-    assert rel(to_np(y), want) < tolerance("bf16", floor)
+    assert rel(to_np(y), want) < tolerance("fp16", floor)
     if emulated_band_holds(Un, Q5, mode):
         assert sigma_band_error(Un, to_np(y), Q5) < 0.05
     else:
@@ -101,13 +114,37 @@ def test_other_coefficient_schedules_and_restart_points():
         assert rel(to_np(y), want) < 2e-2, (mode, ra)
 
 
+@pytest.mark.parametrize("compute,shape", [("fp16", (200, 600)), ("bf16", (300, 900)), ("fp32", (64, 160)),
+                                           ("fp32", (300, 700))])
+@pytest.mark.parametrize("ra,every", [(2, 2), (1, 1), (1, 3)])
+def test_periodic_restarts(compute, shape, ra, every):
+    """The stabilised form restarted after iteration ra and every `every`
+    iterations after it (six quintic iterations): the result matches the
+    oracle's, and the products the library launches add up to the oracle's
+    FLOP count for exactly those restarts (each restart is a pair of
+    rectangular products that a single restart would not run)."""
+    dtype = torch.float32 if compute == "fp32" else torch.bfloat16
+    X = synth.gaussian(*shape, seed=17 + ra + 5 * every, device=DEV, dtype=dtype)
+    coeffs = [oracle.QUINTIC] * 6
+    nsm.muon_profile_begin()
+    (y,), st = gpu_ns([X], coeffs=coeffs, mode="gram_stabilized", restart_after=ra, restart_every=every,
+                      compute_dtype=compute)
+    prof = nsm.muon_profile_end()
+    assert st == [0]
+    want = oracle.newton_schulz(to_np(X), coeffs, mode="gram_stabilized", restart_after=ra, restart_every=every)
+    assert rel(to_np(y), want) < tolerance(compute), (compute, rel(to_np(y), want))
+    launched = sum(r["flops"] for r in prof if r["kernel"] not in ("pack_kernel", "norm_kernel", "unpack_kernel"))
+    assert launched == pytest.approx(oracle.flops(*shape, 6, "gram_stabilized", ra, every), rel=1e-12)
+    assert launched != pytest.approx(oracle.flops(*shape, 6, "gram_stabilized", ra, 0), rel=1e-6)
+
+
 def test_gram_dtype_bf16_option():
     X = synth.gaussian(256, 768, seed=4, device=DEV, dtype=torch.bfloat16)
     for mode in ("gram", "gram_stabilized"):
         (y,), st = gpu_ns([X], mode=mode, gram_dtype="bf16")
         want = oracle.newton_schulz(to_np(X), Q5, mode=mode)
         assert st == [0]
-        assert rel(to_np(y), want) < tolerance("bf16", emulated_floor(to_np(X), Q5, mode, gram_fmt="bf16"))
+        assert rel(to_np(y), want) < tolerance("bf16", emulated_floor(to_np(X), Q5, mode, chain="bf16"))
 
 
 # ---------------------------------------------------------------------------
@@ -222,10 +259,12 @@ def _groups_for_step(spec, w_dtype, seed):
 
 @pytest.mark.parametrize("mode", ["standard", "gram_stabilized"])
 @pytest.mark.parametrize("nesterov", [True, False])
-def test_muon_step_vs_oracle(mode, nesterov):
+@pytest.mark.parametrize("compute", ["fp16", "bf16"])
+def test_muon_step_vs_oracle(mode, nesterov, compute):
     # 2 wide + 1 tall of the same oriented shape (merged batch), a square one, a ragged one
     spec = [(192, 640), (192, 640), (640, 192), (256, 256), (72, 200)]
-    hp = dict(lr=0.05, momentum=0.9, nesterov=nesterov, weight_decay=0.2, scale_coef=0.3, mode=mode)
+    hp = dict(lr=0.05, momentum=0.9, nesterov=nesterov, weight_decay=0.2, scale_coef=0.3, mode=mode,
+              compute_dtype=compute)
     Ws, Gs, Ms = _groups_for_step(spec, torch.float32, 11)
     W0 = [to_np(w) for w in Ws]
     M0 = [to_np(m) for m in Ms]
@@ -240,7 +279,8 @@ def test_muon_step_vs_oracle(mode, nesterov):
         step = 0.05 * 0.3 * math.sqrt(max(r, c))
         O_gpu = ((1 - 0.05 * 0.2) * W0[i] - to_np(Ws[i])) / step
         U = oracle.nesterov_blend(to_np(Gs[i]), Mr, 0.9, nesterov)
-        assert rel(O_gpu, Or) < tolerance("bf16", emulated_floor(U, Q5, mode)), i
+        floor = emulated_floor(U, Q5, mode, chain=chain_of(mode, compute)) if compute == "bf16" else None
+        assert rel(O_gpu, Or) < tolerance(compute, floor), i
         assert sigma_band_error(U, O_gpu, Q5) < 0.05
 
 
@@ -341,7 +381,7 @@ def test_workspace_too_small_is_rejected():
 def test_captured_step_replays_the_eager_step():
     """A step recorded in a CUDA graph and replayed gives the eager step's bits."""
     spec = [(128, 384), (384, 128), (96, 200)]
-    for compute, wdt in (("bf16", torch.bfloat16), ("fp32", torch.float32)):
+    for compute, wdt in (("fp16", torch.bfloat16), ("bf16", torch.bfloat16), ("fp32", torch.float32)):
         Wa, Ga, Ma = _groups_for_step(spec, wdt, 31)
         Wb = [w.clone() for w in Wa]
         Mb = [m.clone() for m in Ma]

@@ -1,7 +1,8 @@
-"""Multi-process host logic on CPU with the gloo backend (world size 2):
+"""Multi-process host logic on CPU with the gloo backend (world size 2-3):
 the bench's cross-rank timing reduction and weak-scaling value, and the
-sharded step's ownership plan and weight exchange (with an injected local
-update in place of the CUDA step)."""
+sharded step's ownership plan and weight exchange, with injected local
+updates in place of the CUDA step: rank-tagged ones that show where each
+weight came from, and the fp64 oracle's own Muon step."""
 import os
 import socket
 
@@ -89,6 +90,43 @@ def _idle_rank_worker(rank, world, port, q):
     dist.destroy_process_group()
 
 
+def _oracle_step_worker(rank, world, port, q):
+    """Each owner runs the method's own update (the fp64 oracle's Muon step on
+    its matrices) as the local step; after the exchange every rank must hold
+    the full set of updated weights that one process computing every matrix
+    gets, and each owner the new momentum of its own matrices."""
+    _init(rank, world, port)
+    import numpy as np
+
+    import oracle
+    import synth
+    hp = dict(lr=0.02, momentum=0.95, nesterov=True, weight_decay=0.1, scale_coef=0.2, eps=1e-7,
+              coeffs=[oracle.QUINTIC] * 5)
+    shapes = [(24, 40), (40, 24), (16, 16), (32, 72), (8, 20)]
+    params = [synth.gaussian(r, c, 10 + i).double() for i, (r, c) in enumerate(shapes)]
+    grads = [synth.gaussian(r, c, 20 + i).double() for i, (r, c) in enumerate(shapes)]
+    moms0 = [synth.gaussian(r, c, 30 + i, std=0.1).double() for i, (r, c) in enumerate(shapes)]
+    want = [oracle.muon_step(p.numpy(), g.numpy(), m.numpy(), **hp) for p, g, m in zip(params, grads, moms0)]
+    owner = lpt_owners([ns_cost(s) for s in shapes], world)
+    moms = {i: moms0[i].clone() for i in range(len(shapes)) if owner[i] == rank}
+
+    def oracle_local(ps, gs, ms, **h):
+        def run():
+            for p, g, m in zip(ps, gs, ms):
+                W, M, _ = oracle.muon_step(p.numpy(), g.numpy(), m.numpy(), **hp)
+                p.copy_(torch.from_numpy(W))
+                m.copy_(torch.from_numpy(M))
+        return run
+
+    step = ShardedMuonStep(params, grads, moms, local_step_factory=oracle_local, **hp)
+    step()
+    ok_w = all(np.array_equal(params[i].numpy(), want[i][0]) for i in range(len(shapes)))
+    ok_m = all(np.array_equal(moms[i].numpy(), want[i][1]) for i in moms)
+    q.put((rank, ok_w and ok_m, owner))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def _spawn(fn, world=2):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
@@ -137,3 +175,9 @@ def test_sharded_step_with_a_rank_that_owns_nothing():
     owned = [o for _, _, o in out]
     assert sorted(i for o in owned for i in o) == [0, 1]
     assert [] in owned
+
+
+def test_sharded_step_exchanges_the_methods_updates():
+    out = _spawn(_oracle_step_worker)
+    assert [ok for _, ok, _ in out] == [True, True]
+    assert sorted(set(out[0][2])) == [0, 1]  # both ranks own matrices
