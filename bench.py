@@ -139,7 +139,7 @@ class ClockSampler:
 
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,clocks.mem")
 
     def __init__(self, device):
         self.uuid = None
@@ -188,8 +188,10 @@ class ClockSampler:
         mx = max(num(r[2]) for r in rows)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        mem = [num(r[9]) for r in rows if len(r) > 9]
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": reasons, "samples": len(rows),
-                "power_w_max": max(num(r[3]) for r in rows)}
+                "power_w_max": max(num(r[3]) for r in rows),
+                "mem_mhz": statistics.median(mem) if mem else None}
 
 
 def kernel_source_hash(kernel: str) -> str | None:
@@ -236,7 +238,7 @@ def roofline_from_profile(prof, peaks, peak_kind, workload=None, compute="fp16")
             continue
         sec = r["ms"] / 1e3
         row = {"kernel": k, "launches": r["launches"], "ms": round(r["ms"], 4)}
-        if k.startswith("tc_product"):
+        if k.startswith("tc_"):
             peak = tf32_peak if k.endswith("[3xtf32]") else bf16_sust
             ex = r.get("exec_flops", r["flops"])
             row.update(bound="tensor", executed_tflops=round(ex / sec / 1e12, 1),

@@ -291,8 +291,8 @@ __global__ void convert_kernel(const void* src, int sdt, void* dst, int ddt, lon
 // ----------------------------------------------------------------------------
 template <typename TS, typename TX>
 static void pack_dispatch2(const PackArgs& a, const SegmentPtrs& p, cudaStream_t s) {
-  dim3 grid(pack_tiles(a.rows, a.cols), a.count);
   const bool trans = a.rows > a.cols;
+  dim3 grid(pack_tiles(a.rows, a.cols), a.count);
   if (a.momentum_mode) {
     if (trans) pack_kernel<TS, TX, true, true><<<grid, kPackThreads, 0, s>>>(a, p);
     else pack_kernel<TS, TX, true, false><<<grid, kPackThreads, 0, s>>>(a, p);

@@ -12,9 +12,10 @@
 //
 // Dependencies are tracked per product and matrix: every epilogue warp of a
 // tile, once its stores have landed in memory, adds one to done[p][b] (release,
-// GPU scope).  A tile of product p for matrix b starts loading only when
-// done[p-1][b] has reached all arrivals of product p-1 for that matrix
-// (acquire).  Product p-1 itself waited for p-2, so every earlier product of
+// GPU scope).  The scheduler publishes a tile of product p for matrix b only
+// when done[p-1][b] has reached all arrivals of product p-1 for that matrix
+// (acquire); the roles that follow it read the tile through the cluster-scope
+// ring, which carries that ordering to them.  Product p-1 itself waited for p-2, so every earlier product of
 // the chain is complete for matrix b, which covers every read-after-write and
 // write-after-read hazard of the chain's buffers.  Tiles are handed out in
 // chain order and the grid is co-resident, so a waiting tile only waits for
@@ -220,7 +221,13 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
                                  cp.timeout_ns))
             break;
           t = held;
-          if (t >= 0) held = take(i + 1);
+          if (t >= 0) {
+            held = take(i + 1);
+            // the tile's operands were written by earlier products of the chain:
+            // acquire them here, once for the whole pair, before publishing it
+            const ChainTile dt = decode_chain(cp, t);
+            if (!dep_ready(dt.prod, dt.t.b)) break;
+          }
           tile_ring[slot] = t;
           st_cluster_s32(mapa(smem_u32(&tile_ring[slot]), 1), t);
           remote_arrive(mapa(smem_u32(&ring_full[slot]), 0));
@@ -231,8 +238,9 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
         if (t < 0) break;
         const ChainTile ct = decode_chain(cp, t);
         const ChainProduct& pr = cp.prod[ct.prod];
-        // the operands of this tile were written by earlier products of the chain
-        if (!dep_ready(ct.prod, ct.t.b)) break;
+        // the leader acquired this tile's inputs before publishing it (below);
+        // the peer synchronised with the leader through the ring, and both
+        // order the acquire before their TMA (async proxy) reads
         fence_proxy_async_global();
         const bool narrow = pr.N - ct.t.TN * 256 <= 128;
         const int row0 = ct.t.TM * 256 + (int)rank * 128;
@@ -316,14 +324,13 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
       const Tile tl{ct.t.b, ct.t.TM * 2 + (int)rank, ct.t.TN};
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      // C was written by an earlier product: the leader acquired it before
+      // publishing this tile, and lane 0 read the tile from the ring with
+      // acquire semantics; the warp barrier orders that before every lane's loads
       int ok = 1;
-      if (lane == 0) {
-        ok = mbar_wait(smem_u32(&tfull_bar[acc]), aph, abort_flag, cp.timeout_ns);
-        // C was written by an earlier product: acquire it here too
-        if (ok && p.C != nullptr) ok = dep_ready(ct.prod, tl.b);
-      }
+      if (lane == 0) ok = mbar_wait(smem_u32(&tfull_bar[acc]), aph, abort_flag, cp.timeout_ns);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      __syncwarp();  // orders lane 0's acquire before every lane's loads of C
+      __syncwarp();
       if (!ok) break;
       tc_fence_after();
       const float f = matrix_scale(p.scale, p.scale_pow, tl.b);
@@ -343,6 +350,11 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
           for (int k = 0; k < 4; ++k) creg[k] = src[k];
           c_ready = true;
         }
+        WPrefetch wpf;
+        wpf.ok = false;
+        if constexpr (UPD) {
+          if (upd) wpf = prefetch_w(p, u, tl, q, lane, c);
+        }
         uint32_t r[32];
         tmem_ld32(tbase + (uint32_t)(c * 32), r);
         if (cc == 3) {
@@ -352,7 +364,7 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
         }
         if constexpr (UPD) {
           if (upd) {
-            update_chunk(p, u, tl, q, lane, c, r, creg, c_ready, f, S);
+            update_chunk(p, u, tl, q, lane, c, r, creg, c_ready, f, S, wpf);
             continue;
           }
         }

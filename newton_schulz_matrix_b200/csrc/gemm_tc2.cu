@@ -290,6 +290,11 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           for (int i = 0; i < 4; ++i) creg[i] = src[i];
           c_ready = true;
         }
+        WPrefetch wpf;
+        wpf.ok = false;
+        if constexpr (UPD) {
+          wpf = prefetch_w(p, u, tl, q, lane, c);
+        }
         uint32_t r[32];
         tmem_ld32(tbase + (uint32_t)(c * 32), r);
         if (cc == 3) {
@@ -298,7 +303,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           if (lane == 0) remote_arrive(leader_tempty + acc * 8);
         }
         if constexpr (UPD) {
-          update_chunk(p, u, tl, q, lane, c, r, creg, c_ready, f, S);
+          update_chunk(p, u, tl, q, lane, c, r, creg, c_ready, f, S, wpf);
         } else {
           epilogue_chunk<SYM>(p, &tmap_d, tl, q, lane, c, r, creg, c_ready, f, S, T);
         }

@@ -327,47 +327,96 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMa
 }
 
 // ------------------------------------------------------------------ fused Muon update
-// Load / update / store 16 consecutive W elements at `w` (16-byte aligned when
-// `vec`; otherwise only the first `valid` are touched, one by one).
-__device__ __forceinline__ void update16(char* w, int wdt, const float* o, int valid, bool vec, float decay,
-                                         float step) {
-  if (vec) {
-    if (wdt == kFP32) {
-      float4* q = reinterpret_cast<float4*>(w);
+// The last product of a Muon step's chain can write W <- decay W - step O
+// itself.  A warp's 32 x 32 box of O is staged in its shared-memory box in W's
+// own orientation (row r of the staging box = row r of the W block the box
+// covers), and the lanes then update W in four passes of 8 rows x 64 bytes:
+// lane L takes row 8 it + L / 4 and its 16-byte segment L % 4, so every access
+// instruction of the warp covers 8 contiguous 64-byte row pieces.
+
+// Where the box of (t, q, chunk) lies in W: its first element, the row pitch,
+// and how many rows and columns of it exist.
+struct WBox {
+  char* base;
+  long long ld;
+  int rows, cols, wdt, es;
+};
+template <typename Slots>
+__device__ __forceinline__ WBox w_box(const Params& p, const Slots& u, const Tile& t, int q, int chunk) {
+  const int gi_base = t.tm * BM + q * 32;
+  const int gj0 = t.tn * BN + chunk * 32;
+  const unsigned kind = u.kind[t.b];
+  WBox w;
+  w.wdt = (int)(kind >> 1);
+  w.es = w.wdt == kFP32 ? 4 : 2;
+  char* W = reinterpret_cast<char*>(u.w[t.b]);
+  if (!(kind & 1u)) {  // W is M x N like O
+    w.ld = p.N;
+    w.base = W + ((long long)gi_base * p.N + gj0) * w.es;
+    w.rows = min(32, p.M - gi_base);
+    w.cols = min(32, p.N - gj0);
+  } else {             // W is N x M: the box's rows are O's columns
+    w.ld = p.M;
+    w.base = W + ((long long)gj0 * p.M + gi_base) * w.es;
+    w.rows = min(32, p.N - gj0);
+    w.cols = min(32, p.M - gi_base);
+  }
+  return w;
+}
+
+// The 16-bit W segments a lane updates (one per pass), loaded ahead of the
+// accumulator read so that their latency overlaps it.
+struct WPrefetch {
+  uint4 q[4];
+  bool ok;
+};
+template <typename Slots>
+__device__ __forceinline__ WPrefetch prefetch_w(const Params& p, const Slots& u, const Tile& t, int q, int lane,
+                                                int chunk) {
+  WPrefetch pf;
+  pf.ok = false;
+  const int gi_base = t.tm * BM + q * 32;
+  const int gj0 = t.tn * BN + chunk * 32;
+  if (gj0 + 32 > p.N || gi_base + 32 > p.M) return pf;  // ragged boxes load W as they go
+  const WBox w = w_box(p, u, t, q, chunk);
+  if (w.wdt == kFP32 || (w.ld * 2) % 16 != 0) return pf;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float4 x = q[k];
-        x.x = weight_update(x.x, o[4 * k], decay, step);
-        x.y = weight_update(x.y, o[4 * k + 1], decay, step);
-        x.z = weight_update(x.z, o[4 * k + 2], decay, step);
-        x.w = weight_update(x.w, o[4 * k + 3], decay, step);
-        q[k] = x;
-      }
-    } else {
-      uint4* q = reinterpret_cast<uint4*>(w);
-      uint4 x[2] = {q[0], q[1]};
-      float v[16];
-      if (wdt == kBF16) {
-        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(x);
+  for (int it = 0; it < 4; ++it)
+    pf.q[it] = *reinterpret_cast<const uint4*>(w.base + ((long long)(it * 8 + (lane >> 2)) * w.ld + (lane & 3) * 8) * 2);
+  pf.ok = true;
+  return pf;
+}
+
+// W[0..valid) <- weight_update(W, o) for 8 consecutive elements at `w`
+// (16-byte aligned when `vec`, then `pre` may hold them already for 16-bit W).
+__device__ __forceinline__ void update8(char* w, int wdt, const float* o, int valid, bool vec, float decay, float step,
+                                        bool have_pre, uint4 pre) {
+  if (vec && wdt == kFP32) {
+    float4* q = reinterpret_cast<float4*>(w);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = weight_update(__bfloat162float(e[k]), o[k], decay, step);
-        __nv_bfloat16* d = reinterpret_cast<__nv_bfloat16*>(x);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) d[k] = __float2bfloat16_rn(v[k]);
-      } else {
-        const __half* e = reinterpret_cast<const __half*>(x);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = weight_update(__half2float(e[k]), o[k], decay, step);
-        __half* d = reinterpret_cast<__half*>(x);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) d[k] = __float2half_rn(v[k]);
-      }
-      q[0] = x[0];
-      q[1] = x[1];
+    for (int k = 0; k < 2; ++k) {
+      float4 x = q[k];
+      x.x = weight_update(x.x, o[4 * k], decay, step);
+      x.y = weight_update(x.y, o[4 * k + 1], decay, step);
+      x.z = weight_update(x.z, o[4 * k + 2], decay, step);
+      x.w = weight_update(x.w, o[4 * k + 3], decay, step);
+      q[k] = x;
     }
+  } else if (vec) {
+    uint4 x = have_pre ? pre : *reinterpret_cast<const uint4*>(w);
+    if (wdt == kBF16) {
+      __nv_bfloat16* e = reinterpret_cast<__nv_bfloat16*>(&x);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) e[k] = __float2bfloat16_rn(weight_update(__bfloat162float(e[k]), o[k], decay, step));
+    } else {
+      __half* e = reinterpret_cast<__half*>(&x);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) e[k] = __float2half_rn(weight_update(__half2float(e[k]), o[k], decay, step));
+    }
+    *reinterpret_cast<uint4*>(w) = x;
   } else {
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
+    for (int k = 0; k < 8; ++k)
       if (k < valid) store_any(w, k, wdt, weight_update(load_any(w, k, wdt), o[k], decay, step));
   }
 }
@@ -375,13 +424,12 @@ __device__ __forceinline__ void update16(char* w, int wdt, const float* o, int v
 // The fused-update counterpart of epilogue_chunk (non-symmetric products):
 // O = f (c_acc acc + c_in C) for this warp's 32 rows x 32 columns, rounded to
 // the chain's type as the stored X would be, then W <- decay W - step O for
-// matrix t.b.  A matrix stored transposed (m x n) goes through this warp's
-// staging box, so that each lane then updates one contiguous W row segment.
-// Non-finite O raises MUON_STATUS_NONFINITE in the matrix's status word.
+// matrix t.b through the staging box S (see above).  Non-finite O raises
+// MUON_STATUS_NONFINITE in the matrix's status word.
 template <typename Slots>
 __device__ __forceinline__ void update_chunk(const Params& p, const Slots& u, const Tile& t, int q, int lane,
                                              int chunk, const uint32_t (&acc)[32], const uint4 (&creg)[4],
-                                             bool c_ready, float f, uint8_t* S) {
+                                             bool c_ready, float f, uint8_t* S, const WPrefetch& pf) {
   const int gi_base = t.tm * BM + q * 32;
   const int gi = gi_base + lane;
   const int gj0 = t.tn * BN + chunk * 32;
@@ -419,40 +467,40 @@ __device__ __forceinline__ void update_chunk(const Params& p, const Slots& u, co
   bad = __any_sync(0xffffffffu, bad);
   if (bad && lane == 0 && u.status != nullptr) atomicOr(u.status + u.status_idx[t.b], kStatusNonFinite);
 
-  const unsigned kind = u.kind[t.b];
-  const int wdt = (int)(kind >> 1);
-  const int es = wdt == kFP32 ? 4 : 2;
-  char* W = reinterpret_cast<char*>(u.w[t.b]);
-  if (!(kind & 1u)) {
-    // W is M x N like O: this lane's row gi, columns gj0 .. gj0 + 31
-    if (gi < p.M) {
-      char* row = W + ((long long)gi * p.N + gj0) * es;
-      const int valid = min(32, p.N - gj0);
-      const bool vec = valid == 32 && ((long long)p.N * es) % 16 == 0;
-      update16(row, wdt, v, min(16, valid), vec, u.decay, u.step);
-      if (valid > 16) update16(row + 16 * es, wdt, v + 16, valid - 16, vec, u.decay, u.step);
-    }
+  const bool trans = (u.kind[t.b] & 1u) != 0;
+  __syncwarp();  // every lane is done with S's previous contents
+  if (!trans) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(S + sw64(lane, k)) = oq[k];
   } else {
-    // W is N x M: transpose the 32 x 32 box of O through shared memory, then
-    // lane L updates W row gj0 + L, columns gi_base .. gi_base + 31
     const uint16_t* ob = reinterpret_cast<const uint16_t*>(oq);
-    __syncwarp();
 #pragma unroll
     for (int j = 0; j < 32; ++j)
       *reinterpret_cast<uint16_t*>(S + sw64(j, lane >> 3) + (lane & 7) * 2) = ob[j];
-    __syncwarp();
-    uint4 tq[4];
+  }
+  __syncwarp();
+  const WBox w = w_box(p, u, t, q, chunk);
+  const bool rows_vec = (w.ld * w.es) % 16 == 0;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) tq[k] = *reinterpret_cast<const uint4*>(S + sw64(lane, k));
-    float o[32];
-    cvt_row32(tq, p.d_dtype, o);
-    if (gj0 + lane < p.N) {
-      char* row = W + ((long long)(gj0 + lane) * p.M + gi_base) * es;
-      const int valid = min(32, p.M - gi_base);
-      const bool vec = valid == 32 && ((long long)p.M * es) % 16 == 0;
-      update16(row, wdt, o, min(16, valid), vec, u.decay, u.step);
-      if (valid > 16) update16(row + 16 * es, wdt, o + 16, valid - 16, vec, u.decay, u.step);
+  for (int it = 0; it < 4; ++it) {
+    const int r = it * 8 + (lane >> 2);
+    const int c0 = (lane & 3) * 8;
+    if (r >= w.rows || c0 >= w.cols) continue;
+    const int valid = min(8, w.cols - c0);
+    // this lane's 8 values of O: row r of the staging box, 16-byte chunk lane % 4
+    const uint4 oseg = *reinterpret_cast<const uint4*>(S + sw64(r, lane & 3));
+    float o[8];
+    if (p.d_dtype == kBF16) {
+      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&oseg);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] = __bfloat162float(e[k]);
+    } else {
+      const __half* e = reinterpret_cast<const __half*>(&oseg);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[k] = __half2float(e[k]);
     }
+    update8(w.base + ((long long)r * w.ld + c0) * w.es, w.wdt, o, valid, valid == 8 && rows_vec, u.decay, u.step,
+            pf.ok, pf.q[it]);
   }
 }
 

@@ -79,3 +79,13 @@ def test_streamed_slices_take_the_widest_short_side_first_and_respect_the_budget
         assert len(sl) == 1 or sum(nbytes[i] for i in sl) <= 64 << 20
     assert [len(sl) for sl in slices] == [1, 1, 2, 3]             # 29 MB experts pair up (the small one joins); 264 MB dense alone
     assert plan_slices([], [], 1) == []
+
+
+def test_a_chain_launch_is_a_tensor_class_of_its_own():
+    prof = [_prof("pack_kernel", 6, 30.0, 0.0, nbytes=118.9e9),
+            _prof("tc_chain", 3, 380.0, 513e12, exec_flops=420e12),
+            _prof("status_or_kernel", 6, 0.1, 0.0, nbytes=1e3)]
+    r = bench.roofline_from_profile(prof, PEAKS, "measured", "kimi-k2", "fp16")
+    assert r["kernel"] == "tc_chain"
+    assert r["achieved"] == pytest.approx(420e12 / 0.380 / 1e12, rel=1e-3)
+    assert r["algorithmic_tflops"] == pytest.approx(513e12 / 0.380 / 1e12, rel=1e-3)

@@ -1,17 +1,17 @@
 """The library's launch modes give the same bits.
 
-By default a 16-bit chain whose short side is at least 256 runs as one
-persistent launch per chunk (products ordered by per-matrix dependency
-counters, gemm_chain.cu), the Muon update is written by the last product's
-epilogue, and product launches may overlap the previous kernel's drain.
-Each of these can be switched off when the library loads (MUON_CHAIN=0,
-MUON_FUSED_UPDATE=0, MUON_PDL=0), and tiles can be handed out in a fixed
-round-robin order instead of from the counter (MUON_TILE_ORDER=static): the
-tests run every case in a child process
-with a switch off and compare W, M, X and the status words bit for bit with
-the default run in this process.  The arithmetic is the same in every mode
-(same tiles, same k order, same epilogue, the update's rounding pinned), so
-any difference is a scheduling or memory-ordering fault.
+The product launches of a chain can go out one by one (the default: tiles
+from a per-launch counter, programmatic dependent launch) or as one
+persistent launch per chunk (MUON_CHAIN=1: products ordered by per-matrix
+dependency counters, gemm_chain.cu); the Muon update can be written by the
+last product's epilogue or by a separate pass (MUON_FUSED_UPDATE); launches
+may or may not overlap the previous kernel's drain (MUON_PDL=0); tiles can be
+handed out round-robin instead of from the counter (MUON_TILE_ORDER=static).
+Each switch is read when the library loads, so the tests run every case in
+a child process per variant and compare W, M, X and the status words bit for
+bit with the default run in this process.  The arithmetic is the same in
+every mode (same tiles, same k order, same epilogue, the update's rounding
+pinned), so any difference is a scheduling or memory-ordering fault.
 
 Cases: wide and tall matrices merged in one batch, ragged shapes whose rows
 are not 16-byte multiples, every W dtype, all three forms, a non-finite
@@ -80,24 +80,22 @@ def _bits(t):
     return t.view({1: torch.int8, 2: torch.int16, 4: torch.int32}[t.element_size()])
 
 
-def _in_child(name, env_off, path):
+def _in_child(name, env, path):
     code = ("import sys, torch; sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r});"
             "import test_gpu_launch_modes as t; torch.save(t.run_case({name!r}), {path!r})").format(
         root=ROOT, tests=os.path.join(ROOT, "tests"), name=name, path=path)
-    env = dict(os.environ, **{k: ("static" if k == "MUON_TILE_ORDER" else "0") for k in env_off})
-    subprocess.run([sys.executable, "-c", code], check=True, env=env, cwd=ROOT, timeout=600)
+    subprocess.run([sys.executable, "-c", code], check=True, env=dict(os.environ, **env), cwd=ROOT, timeout=600)
     return torch.load(path)
 
 
-SWITCHES = [("MUON_CHAIN",), ("MUON_FUSED_UPDATE",), ("MUON_PDL",), ("MUON_CHAIN", "MUON_FUSED_UPDATE", "MUON_PDL"),
-            ("MUON_TILE_ORDER",)]
+SWITCHES = [{"MUON_CHAIN": "1"}, {"MUON_FUSED_UPDATE": "0"}, {"MUON_FUSED_UPDATE": "1"}, {"MUON_PDL": "0"},
+            {"MUON_TILE_ORDER": "static"}, {"MUON_CHAIN": "1", "MUON_FUSED_UPDATE": "1", "MUON_PDL": "0"}]
+MODE_VARS = ("MUON_CHAIN", "MUON_FUSED_UPDATE", "MUON_PDL", "MUON_TILE_ORDER")
 
 
 @pytest.mark.parametrize("name", sorted(STEP_CASES) + sorted(NS_CASES))
 def test_every_launch_mode_gives_the_same_bits(name):
-    for k in ("MUON_CHAIN", "MUON_FUSED_UPDATE", "MUON_PDL"):
-        assert os.environ.get(k, "1") != "0"
-    assert os.environ.get("MUON_TILE_ORDER", "dynamic") != "static"
+    assert not any(k in os.environ for k in MODE_VARS)  # this process runs the defaults
     got, st = run_case(name)
     if name in STEP_CASES and "nan" in STEP_CASES[name]:
         bad = STEP_CASES[name]["nan"]
@@ -105,22 +103,23 @@ def test_every_launch_mode_gives_the_same_bits(name):
     else:
         assert st.tolist() == [0] * len(st)
     with tempfile.TemporaryDirectory() as d:
-        for i, off in enumerate(SWITCHES):
-            ref, st0 = _in_child(name, off, os.path.join(d, f"ref{i}.pt"))
-            assert torch.equal(st, st0), off
+        for i, env in enumerate(SWITCHES):
+            ref, st0 = _in_child(name, env, os.path.join(d, f"ref{i}.pt"))
+            assert torch.equal(st, st0), env
             for a, b in zip(got, ref):
-                assert a.dtype == b.dtype and torch.equal(_bits(a), _bits(b)), off
+                assert a.dtype == b.dtype and torch.equal(_bits(a), _bits(b)), env
 
 
-def test_default_step_has_no_unpack_pass_and_one_chain_launch():
-    """The profile of a default 16-bit step: one chain launch per chunk, no
-    unpack_kernel (the update is in the last product's epilogue)."""
+def test_profile_of_a_default_step():
+    """A default 16-bit step launches its products separately (no chain) and
+    runs the update as configured by default."""
     W = [synth.gaussian(512, 1024, 5, "cuda").bfloat16()]
     G = [synth.gaussian(512, 1024, 6, "cuda").bfloat16()]
     M = [torch.zeros(512, 1024, device="cuda")]
     nsm.muon_profile_begin()
     nsm.muon_step(W, G, M)
     prof = {r["kernel"]: r for r in nsm.muon_profile_end()}
-    assert "unpack_kernel" not in prof and "tc_product" not in prof
-    assert prof["tc_chain"]["launches"] == 1
-    assert prof["tc_chain"]["flops"] == pytest.approx(nsm.muon_ns_flops(512, 1024), rel=1e-12)
+    assert "tc_chain" not in prof
+    assert prof["tc_product"]["launches"] == 5 and prof["tc_product[symmetric]"]["launches"] == 10
+    flops = prof["tc_product"]["flops"] + prof["tc_product[symmetric]"]["flops"]
+    assert flops == pytest.approx(nsm.muon_ns_flops(512, 1024), rel=1e-12)
