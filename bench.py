@@ -53,7 +53,10 @@ KERNEL_SOURCES = {
 # written per launch, averaged over the launches of one step, from an ncu
 # launch list of `python bench.py --workload <w> --compute <c> --steps 1
 # --warmup 1` with --metrics dram__bytes_read.sum,dram__bytes_write.sum).
-MEASURED_TRAFFIC: dict = {}
+MEASURED_TRAFFIC: dict = {
+    ("kimi-k2", "fp16", "tc_product"): ("94d115be38917e3e", 17.46e9),
+    ("kimi-k2", "fp16", "tc_product[symmetric]"): ("94d115be38917e3e", 6.89e9),
+}
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
@@ -75,8 +78,9 @@ def parse_args():
     p.add_argument("--sharded", action="store_true",
                    help="strong scaling: shard one workload across the ranks (ownership by NS FLOPs, owner "
                         "broadcast of the updated weights) instead of one full workload per rank")
-    p.add_argument("--report", choices=["stress"], default=None,
-                   help="stress: the ill-conditioned sweep (one JSON line per (n, alpha) point) instead of the bench")
+    p.add_argument("--report", choices=["stress", "parity"], default=None,
+                   help="stress: the ill-conditioned sweep (one JSON line per (n, alpha) point); parity: errors "
+                        "against the fp64 oracle on sampled matrices of each workload, every form")
     return p.parse_args()
 
 
@@ -395,10 +399,79 @@ def run_stress_report(args):
             torch.cuda.empty_cache()
 
 
+def run_parity_report(args):
+    """Errors against the fp64 oracle at the workloads' full sizes: each
+    workload runs as one Muon step in the bench's launch configuration (fp32
+    copies of W, so that O = (decay W0 - W1) / step is exact), and sampled
+    matrices are compared with oracle.muon_step.  One JSON line per (workload,
+    form, compute type, matrix): relative Frobenius error, the oracle's
+    stored-precision floor for that chain, sigma-band deviation, oracle time."""
+    import numpy as np
+    import newton_schulz_matrix_b200 as nsm
+    import oracle
+    import synth
+    dev = torch.device("cuda", 0)
+    hp = dict(lr=0.02, momentum=0.95, nesterov=True, weight_decay=0.1, scale_coef=0.2, eps=1e-7,
+              coeffs=[synth.QUINTIC] * 5)
+
+    def floor_of(U, mode, chain):
+        X, _ = oracle.orient(U)
+        f = 1.0 / (oracle.frobenius_norm(X) + hp["eps"])
+        exact = oracle.ns_standard(X * f, hp["coeffs"]) if mode == "standard" else oracle.ns_gram(
+            X * f, hp["coeffs"], 0 if mode == "gram" else 2)
+        start, pre = (oracle.round_to(X, "bf16"), f) if chain == "bf16" else (oracle.round_to(X * f, chain), None)
+        emu = (oracle.ns_standard_stored(start, hp["coeffs"], chain, prescale=pre) if mode == "standard" else
+               oracle.ns_gram_stored(start, hp["coeffs"], chain, 0 if mode == "gram" else 2, prescale=pre))
+        return float(np.linalg.norm(emu - exact) / np.linalg.norm(exact)) if np.all(np.isfinite(emu)) else None
+
+    cases = [("dense-64x1024x4096", lambda: synth.dense_projection(device=dev), [0, 1]),
+             ("moe-64e", lambda: synth.moe_layer(device=dev), None),
+             ("kimi-k2 experts (8 up/gate + 4 down of the set)", lambda: synth.kimi_k2(device=dev, counts=[8, 4, 0, 0]),
+              None)]
+    for name, make, pick in cases:
+        for mode, compute in (("standard", "fp16"), ("standard", "bf16"), ("gram", "fp16"), ("gram_stabilized", "fp16")):
+            w = make()
+            params, grads, moms, samples = [], [], [], []
+            for g in w.groups:
+                samples.append(len(params))
+                params += [x.float() for x in g.W]
+                grads += g.G
+                moms += g.M
+            if pick is not None:
+                samples = pick
+            W0 = {i: params[i].double().cpu().numpy() for i in samples}
+            M0 = {i: moms[i].double().cpu().numpy() for i in samples}
+            step = nsm.MuonStep(params, grads, moms, mode=mode, compute_dtype=compute, **hp)
+            step()
+            torch.cuda.synchronize()
+            status = int((step.status != 0).sum())
+            for i in samples:
+                r, c = params[i].shape
+                G = grads[i].double().cpu().numpy()
+                t0 = time.perf_counter()
+                Wr, Mr, Or = oracle.muon_step(W0[i], G, M0[i], mode=mode, restart_after=2, **hp)
+                oms = (time.perf_counter() - t0) * 1e3
+                sc = hp["lr"] * hp["scale_coef"] * math.sqrt(max(r, c))
+                O = ((1 - hp["lr"] * hp["weight_decay"]) * W0[i] - params[i].double().cpu().numpy()) / sc
+                U = oracle.nesterov_blend(G, Mr, hp["momentum"], True)
+                err = float(np.linalg.norm(O - Or) / np.linalg.norm(Or))
+                chain = compute if mode == "standard" else "fp16"
+                band = sigma_band_device(torch.from_numpy(U).to(dev), torch.from_numpy(O).to(dev), hp["coeffs"])
+                print(json.dumps({"report": "parity", "workload": name, "mode": mode, "compute": compute,
+                                  "shape": [r, c], "rel_err": err, "floor": floor_of(U, mode, chain),
+                                  "sigma_band_dev": band, "status_nonzero": status,
+                                  "oracle_ms": round(oms, 1)}), flush=True)
+            del step, params, grads, moms, w
+            torch.cuda.empty_cache()
+
+
 def main():
     args = parse_args()
     if args.report == "stress":
         run_stress_report(args)
+        return
+    if args.report == "parity":
+        run_parity_report(args)
         return
     if args.impl == "reference":
         run_reference(args)

@@ -185,9 +185,17 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
   auto next_tile = [&](int i, int& t) -> bool {
     const int slot = i % RING;
     const uint32_t rph = (uint32_t)(i / RING) & 1u;
-    if (!mbar_wait_cluster(smem_u32(&ring_full[slot]), rph, abort_flag, cp.timeout_ns)) return false;
-    t = tile_ring[slot];
-    remote_arrive(leader_ring_empty + slot * 8);
+    if (leader) {
+      // the ring and its barriers are this CTA's own: CTA-scope wait and arrive
+      if (!mbar_wait(smem_u32(&ring_full[slot]), rph, abort_flag, cp.timeout_ns)) return false;
+      t = tile_ring[slot];
+      mbar_arrive(smem_u32(&ring_empty[slot]));
+    } else {
+      // published from the leader CTA: cluster-scope acquire, remote release
+      if (!mbar_wait_cluster(smem_u32(&ring_full[slot]), rph, abort_flag, cp.timeout_ns)) return false;
+      t = tile_ring[slot];
+      remote_arrive(leader_ring_empty + slot * 8);
+    }
     return true;
   };
   // The arrivals that mark product p's tiles of matrix b complete.
@@ -230,8 +238,8 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
           }
           tile_ring[slot] = t;
           st_cluster_s32(mapa(smem_u32(&tile_ring[slot]), 1), t);
-          remote_arrive(mapa(smem_u32(&ring_full[slot]), 0));
-          remote_arrive(mapa(smem_u32(&ring_full[slot]), 1));
+          mbar_arrive(smem_u32(&ring_full[slot]));            // this CTA's roles
+          remote_arrive(mapa(smem_u32(&ring_full[slot]), 1));  // the peer's
         } else if (!next_tile(i, t)) {
           break;
         }
@@ -360,7 +368,10 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
         if (cc == 3) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) remote_arrive(leader_tempty + acc * 8);
+          if (lane == 0) {
+            if (leader) mbar_arrive(smem_u32(&tempty_bar[acc]));
+            else remote_arrive(leader_tempty + acc * 8);
+          }
         }
         if constexpr (UPD) {
           if (upd) {

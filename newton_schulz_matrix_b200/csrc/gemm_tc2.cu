@@ -148,9 +148,17 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
   auto next_tile = [&](int i, int& t) -> bool {
     const int slot = i % RING;
     const uint32_t rph = (uint32_t)(i / RING) & 1u;
-    if (!mbar_wait_cluster(smem_u32(&ring_full[slot]), rph, abort_flag, p.timeout_ns)) return false;
-    t = tile_ring[slot];
-    remote_arrive(leader_ring_empty + slot * 8);
+    if (leader) {
+      // the ring and its barriers are this CTA's own: CTA-scope wait and arrive
+      if (!mbar_wait(smem_u32(&ring_full[slot]), rph, abort_flag, p.timeout_ns)) return false;
+      t = tile_ring[slot];
+      mbar_arrive(smem_u32(&ring_empty[slot]));
+    } else {
+      // published from the leader CTA: cluster-scope acquire, remote release
+      if (!mbar_wait_cluster(smem_u32(&ring_full[slot]), rph, abort_flag, p.timeout_ns)) return false;
+      t = tile_ring[slot];
+      remote_arrive(leader_ring_empty + slot * 8);
+    }
     return true;
   };
 
@@ -181,8 +189,8 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           if (t >= 0) held = take(i + 1);
           tile_ring[slot] = t;
           st_cluster_s32(mapa(smem_u32(&tile_ring[slot]), 1), t);
-          remote_arrive(mapa(smem_u32(&ring_full[slot]), 0));
-          remote_arrive(mapa(smem_u32(&ring_full[slot]), 1));
+          mbar_arrive(smem_u32(&ring_full[slot]));            // this CTA's roles
+          remote_arrive(mapa(smem_u32(&ring_full[slot]), 1));  // the peer's
         } else if (!next_tile(i, t)) {
           break;
         }
@@ -300,7 +308,10 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
         if (cc == 3) {
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) remote_arrive(leader_tempty + acc * 8);
+          if (lane == 0) {
+            if (leader) mbar_arrive(smem_u32(&tempty_bar[acc]));
+            else remote_arrive(leader_tempty + acc * 8);
+          }
         }
         if constexpr (UPD) {
           update_chunk(p, u, tl, q, lane, c, r, creg, c_ready, f, S, wpf);
