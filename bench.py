@@ -54,8 +54,8 @@ KERNEL_SOURCES = {
 # launch list of `python bench.py --workload <w> --compute <c> --steps 1
 # --warmup 1` with --metrics dram__bytes_read.sum,dram__bytes_write.sum).
 MEASURED_TRAFFIC: dict = {
-    ("kimi-k2", "fp16", "tc_product"): ("94d115be38917e3e", 17.46e9),
-    ("kimi-k2", "fp16", "tc_product[symmetric]"): ("94d115be38917e3e", 6.89e9),
+    ("kimi-k2", "fp16", "tc_product"): ("f676e32535567062", 17.44e9),
+    ("kimi-k2", "fp16", "tc_product[symmetric]"): ("f676e32535567062", 7.14e9),
 }
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
