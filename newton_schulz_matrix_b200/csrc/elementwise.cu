@@ -8,10 +8,12 @@
 //   step 3 (s(W) = sqrt(max(d_out, d_in))), step 4 and "Innovation 1"
 //   (W = (1 - eta lambda) W - eta U), and the listing's orientation (m <= n).
 //
-// Layout: a 64 x 64 storage tile per 256-thread block; each thread owns 16
-// consecutive elements of one tile row (128-bit loads and stores on the fast
-// path).  Tall matrices go through a padded shared-memory tile so that both
-// the storage read and the oriented write stay row-contiguous.
+// Layout: a 64 x 64 storage tile per 256-thread block.  The pack gives each
+// thread 4 consecutive elements of 4 tile rows (16 threads per 64-element row
+// segment); the update pass gives each thread 16 consecutive elements of one
+// tile row (it measured faster that way).  Tall matrices go through a padded
+// shared-memory tile so that both the storage read and the oriented write
+// stay row-contiguous.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,6 +24,32 @@ constexpr int kPackThreads = 256;
 
 int pack_tiles(int rows, int cols) {
   return ((rows + kTile - 1) / kTile) * ((cols + kTile - 1) / kTile);
+}
+
+template <typename T>
+__device__ __forceinline__ void load4(const T* p, float* v) {
+  // 4 elements: p is 8-byte aligned for 16-bit types, 16-byte aligned for fp32
+  if constexpr (sizeof(T) == 2) {
+    const uint2 q = *reinterpret_cast<const uint2*>(p);
+    const T* e = reinterpret_cast<const T*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = to_f32(e[i]);
+  } else {
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+  }
+}
+template <typename T>
+__device__ __forceinline__ void store4(T* p, const float* v) {
+  if constexpr (sizeof(T) == 2) {
+    uint2 q;
+    T* e = reinterpret_cast<T*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) e[i] = from_f32<T>(v[i]);
+    *reinterpret_cast<uint2*>(p) = q;
+  } else {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  }
 }
 
 template <typename T>
@@ -77,6 +105,13 @@ __device__ __forceinline__ float block_sum_fixed(float v, float* red) {
 // ----------------------------------------------------------------------------
 // pack: U -> oriented workspace X (+ momentum update), sums of squares per tile
 // ----------------------------------------------------------------------------
+// Thread mapping: 16 threads per 64-element row segment, 4 elements each, four
+// row passes of 16 rows.  Every load and store instruction of a warp then
+// covers two whole row segments (2 x 128 bytes of a 16-bit type, 2 x 256 bytes
+// of fp32), so no L1 sector is requested twice.  (With 4 threads per segment
+// and 16 elements each, consecutive 16-byte accesses of a thread each touched
+// half of a sector: half the L1 requests were repeats, and the pack slowed with
+// the SM clock under the power cap.)
 template <typename TS, typename TX, bool MOMENTUM, bool TRANS>
 __global__ void __launch_bounds__(kPackThreads)
 pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
@@ -85,54 +120,65 @@ pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
   const int b = blockIdx.y;
   const int tcols = (a.cols + kTile - 1) / kTile;
   const int r0 = (blockIdx.x / tcols) * kTile, c0 = (blockIdx.x % tcols) * kTile;
-  const int lr = threadIdx.x >> 2, lc = (threadIdx.x & 3) * 16;
-  const int r = r0 + lr;
+  const int lr = threadIdx.x >> 4, lc = (threadIdx.x & 15) * 4;
   const TS* src = reinterpret_cast<const TS*>(p.src[b]);
   float* mom = MOMENTUM ? p.mom[b] : nullptr;
   TX* x = reinterpret_cast<TX*>(a.x) + (long long)b * a.x_batch_stride;
 
   const bool full = (r0 + kTile <= a.rows) && (c0 + kTile <= a.cols) && (a.cols % 8 == 0);
   const bool store = a.pass != 1;
-  float u[16];
-  float ssq = 0.f;
+  float u[4][4];  // [row pass][element]
   if (full) {
-    const long long off = (long long)r * a.cols + c0 + lc;
-    float g[16];
-    load16(src + off, g);
-    if (MOMENTUM) {
-      float m[16];
-      load16(mom + off, m);
+    // every load of the four passes first: one memory round trip per thread
+    float g[4][4], m[4][4];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        m[i] = a.mu * m[i] + (1.f - a.mu) * g[i];
-        u[i] = a.nesterov ? (1.f - a.mu) * g[i] + a.mu * m[i] : m[i];
+    for (int q = 0; q < 4; ++q) {
+      const long long off = (long long)(r0 + q * 16 + lr) * a.cols + c0 + lc;
+      load4(src + off, g[q]);
+      if (MOMENTUM) load4(mom + off, m[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (MOMENTUM) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          m[q][i] = a.mu * m[q][i] + (1.f - a.mu) * g[q][i];
+          u[q][i] = a.nesterov ? (1.f - a.mu) * g[q][i] + a.mu * m[q][i] : m[q][i];
+        }
+        if (store) store4(mom + (long long)(r0 + q * 16 + lr) * a.cols + c0 + lc, m[q]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) u[q][i] = g[q][i];
       }
-      if (store) store16(mom + off, m);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) u[i] = g[i];
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int c = c0 + lc + i;
-      u[i] = 0.f;
-      if (r < a.rows && c < a.cols) {
-        const long long off = (long long)r * a.cols + c;
-        float g = to_f32(src[off]);
-        if (MOMENTUM) {
-          float m = a.mu * mom[off] + (1.f - a.mu) * g;
-          if (store) mom[off] = m;
-          u[i] = a.nesterov ? (1.f - a.mu) * g + a.mu * m : m;
-        } else {
-          u[i] = g;
+    for (int q = 0; q < 4; ++q) {
+      const int r = r0 + q * 16 + lr;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = c0 + lc + i;
+        u[q][i] = 0.f;
+        if (r < a.rows && c < a.cols) {
+          const long long off = (long long)r * a.cols + c;
+          const float gv = to_f32(src[off]);
+          if (MOMENTUM) {
+            const float mv = a.mu * mom[off] + (1.f - a.mu) * gv;
+            if (store) mom[off] = mv;
+            u[q][i] = a.nesterov ? (1.f - a.mu) * gv + a.mu * mv : mv;
+          } else {
+            u[q][i] = gv;
+          }
         }
       }
     }
   }
+  float ssq = 0.f;
   if (a.pass != 2) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) ssq += u[i] * u[i];
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) ssq += u[q][i] * u[q][i];
   }
   if (a.pass == 1) {
     const float s = block_sum_fixed(ssq, red);
@@ -142,34 +188,45 @@ pack_kernel(const PackArgs a, const __grid_constant__ SegmentPtrs p) {
   if (a.pass == 2) {
     const float f = a.scale[b];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) u[i] *= f;
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) u[q][i] *= f;
   }
 
   if (!TRANS) {
     // oriented == storage: row r, columns c0 + lc ...
-    if (full) {
-      store16(x + (long long)r * a.ld_x + c0 + lc, u);
-    } else if (r < a.rows) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (c0 + lc + i < a.cols) x[(long long)r * a.ld_x + c0 + lc + i] = from_f32<TX>(u[i]);
+    for (int q = 0; q < 4; ++q) {
+      const int r = r0 + q * 16 + lr;
+      if (full) {
+        store4(x + (long long)r * a.ld_x + c0 + lc, u[q]);
+      } else if (r < a.rows) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (c0 + lc + i < a.cols) x[(long long)r * a.ld_x + c0 + lc + i] = from_f32<TX>(u[q][i]);
+      }
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) tile[lr][lc + i] = u[i];
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tile[q * 16 + lr][lc + i] = u[q][i];
     __syncthreads();
-    // oriented row j = storage column c0 + lr; oriented columns = storage rows r0 + lc + i
-    const int j = c0 + lr;
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = tile[lc + i][lr];
+    // oriented row j = storage column c0 + q * 16 + lr; oriented columns = storage rows r0 + lc + i
     const bool fullT = (c0 + kTile <= a.cols) && (r0 + kTile <= a.rows);
-    if (fullT) {
-      store16(x + (long long)j * a.ld_x + r0 + lc, v);
-    } else if (j < a.cols) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        if (r0 + lc + i < a.rows) x[(long long)j * a.ld_x + r0 + lc + i] = from_f32<TX>(v[i]);
+    for (int q = 0; q < 4; ++q) {
+      const int j = c0 + q * 16 + lr;
+      float v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) v[i] = tile[lc + i][q * 16 + lr];
+      if (fullT) {
+        store4(x + (long long)j * a.ld_x + r0 + lc, v);
+      } else if (j < a.cols) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (r0 + lc + i < a.rows) x[(long long)j * a.ld_x + r0 + lc + i] = from_f32<TX>(v[i]);
+      }
     }
   }
   if (a.pass == 0) {
