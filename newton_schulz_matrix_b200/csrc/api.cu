@@ -38,13 +38,14 @@ inline int round8(int v) { return (v + 7) / 8 * 8; }
 // ------------------------------------------------------------------ profiler
 enum ProfKind {
   kProfPack, kProfNorm, kProfSyrkTc, kProfGemmTc, kProfGemmSimt, kProfUnpack, kProfFusedSmall, kProfTf32, kProfChain,
-  kProfStatus, kProfKinds
+  kProfStatus, kProfSplit, kProfKinds
 };
 // product kinds cover both tensor-core kernels (gemm_pair_kernel for M >= 256, gemm_kernel below);
 // tc_chain is a whole chain in one launch (gemm_chain_kernel)
 const char* const kProfNames[kProfKinds] = {"pack_kernel", "norm_kernel", "tc_product[symmetric]", "tc_product",
                                             "gemm_simt_kernel", "unpack_kernel", "ns_fused_small_kernel",
-                                            "tc_product[3xtf32]", "tc_chain", "status_or_kernel"};
+                                            "tc_product[3xtf32]", "tc_chain", "status_or_kernel",
+                                            "split_tf32_kernel"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -101,9 +102,12 @@ struct Layout {       // per-chunk workspace layout for a batch
   int n_counters;     // tile-scheduler words: one per product launch of the chain
   size_t head;        // error word + counters, zeroed at the start of each chunk
                       // (followed by the chain launches' done counters: n_counters per matrix)
+  bool tf32;          // fp32 chain on the tensor cores: TF32 hi/lo planes of the operands
   size_t per_matrix;  // bytes per matrix (all buffers)
   size_t fixed;       // bytes independent of the chunk size
 };
+
+bool fp32_tensor_cores();
 
 bool ns_params_ok(const muon_ns_params* ns) {
   if (!ns || ns->iters < 1 || ns->iters > 1000 || !ns->coeffs) return false;
@@ -139,6 +143,14 @@ Layout make_layout(int n, int m, const muon_ns_params* ns) {
   L.per_matrix = 2 * (size_t)n * L.ld_m * L.x_es + (size_t)L.n_sq * n * L.ld_n * L.g_es + (size_t)L.tiles * 4 + 4 +
                  (size_t)L.n_counters * 4;
   L.fixed = kAlign * (2 + L.n_sq + 3) + kAlign + L.head;  // alignment slack + error word and counters
+  // every product of an fp32 chain with n >= 256 runs as 3xTF32 and reads its
+  // operands as hi / lo planes: one X-sized pair and two n x n pairs (a
+  // product has at most two distinct operands, and at most one is X-sized)
+  L.tf32 = ns->compute_dtype == MUON_FP32 && n >= 256 && fp32_tensor_cores();
+  if (L.tf32) {
+    L.per_matrix += 2 * ((size_t)n * L.ld_m + 2 * (size_t)n * L.ld_n) * 4;
+    L.fixed += kAlign * 6;
+  }
   return L;
 }
 
@@ -147,6 +159,8 @@ size_t chunk_bytes(const Layout& L, int chunk) { return L.fixed + L.per_matrix *
 struct Bufs {
   void* X[2];
   void* S[5];
+  float* planes[3][2];  // fp32 tensor-core chains: [X-sized, n x n, n x n][hi, lo]
+  size_t plane_elems[3];
   float* partials;
   float* inv;
   int* err;
@@ -178,6 +192,16 @@ Bufs carve(const Layout& L, int chunk, void* ws) {
   B.partials = reinterpret_cast<float*>(p);
   p += align_up((size_t)chunk * L.tiles * 4, kAlign);
   B.inv = reinterpret_cast<float*>(p);
+  p += align_up((size_t)chunk * 4, kAlign);
+  if (L.tf32) {
+    for (int i = 0; i < 3; ++i) {
+      B.plane_elems[i] = (size_t)chunk * (i == 0 ? B.x_bs : B.s_bs);
+      for (int h = 0; h < 2; ++h) {
+        B.planes[i][h] = reinterpret_cast<float*>(p);
+        p += align_up(B.plane_elems[i] * 4, kAlign);
+      }
+    }
+  }
   return B;
 }
 
@@ -200,6 +224,17 @@ std::vector<Batch> plan_groups(const muon_group* groups, int n_groups) {
 }
 
 // ------------------------------------------------------------------ products
+// The TF32 hi / lo planes of the chunk's fp32 operands, and which buffer's
+// split each pair holds now: a split is reused until a product overwrites its
+// source (X's split serves both X X^T and the update X <- aX + BX).
+struct PlaneCache {
+  float* hi[3] = {};
+  float* lo[3] = {};
+  size_t cap[3] = {};            // elements
+  const void* held[3] = {};      // source buffer of the split the pair holds, or null
+  int n = 0;
+};
+
 struct Ctx {
   int compute;   // MUON_BF16 / MUON_FP16 / MUON_FP32
   cudaStream_t s;
@@ -208,7 +243,28 @@ struct Ctx {
   int n_counters;
   int* used;           // how many of them the chain has taken so far
   std::vector<GemmDesc>* record = nullptr;  // chain mode: collect the products instead of launching them
+  PlaneCache* planes = nullptr;             // fp32 tensor-core chains
 };
+
+// The plane pair that holds (or is to receive) the split of `src`, `elems`
+// values, not pair `avoid` (-1: none).  *fresh: the pair must be (re)written.
+int plane_pair(PlaneCache& pc, const void* src, size_t elems, int avoid, bool* fresh) {
+  for (int i = 0; i < pc.n; ++i)
+    if (i != avoid && pc.held[i] == src && pc.cap[i] >= elems) {
+      *fresh = false;
+      return i;
+    }
+  int best = -1;
+  for (int i = 0; i < pc.n; ++i) {
+    if (i == avoid || pc.cap[i] < elems) continue;
+    // an empty pair first, then the smallest that fits
+    if (best < 0 || (pc.held[i] == nullptr && pc.held[best] != nullptr) ||
+        ((pc.held[i] == nullptr) == (pc.held[best] == nullptr) && pc.cap[i] < pc.cap[best]))
+      best = i;
+  }
+  *fresh = true;
+  return best;
+}
 
 // fp32 products with 256 or more rows run as 3xTF32 on the tensor cores;
 // MUON_FP32_TC=0 keeps every fp32 product on the SIMT kernel.
@@ -235,8 +291,40 @@ int gemm(const Ctx& c, GemmDesc g) {
   const bool prof = profiler().on;
   if (c.compute == MUON_FP32) {
     if (g.M >= 256 && fp32_tensor_cores()) {
-      ProfScope ps(kProfTf32, flops, bytes, c.s, prof ? gemm_tf32x3_exec_flops(g) : 0.0);
-      return gemm_tf32x3(g, c.s);
+      if (c.planes == nullptr) return (int)cudaErrorInvalidValue;
+      PlaneCache& pc = *c.planes;
+      const size_t a_elems = (size_t)g.a_bs * g.batch, b_elems = (size_t)g.b_bs * g.batch;
+      bool fresh_a = false, fresh_b = false;
+      const int ia = plane_pair(pc, g.A, a_elems, -1, &fresh_a);
+      if (ia < 0) return (int)cudaErrorInvalidValue;
+      if (fresh_a) pc.held[ia] = nullptr;  // being rewritten
+      int ib = ia;
+      if (g.B != g.A) {
+        ib = plane_pair(pc, g.B, b_elems, ia, &fresh_b);
+        if (ib < 0) return (int)cudaErrorInvalidValue;
+        if (fresh_b) pc.held[ib] = nullptr;
+      }
+      int rc;
+      if (fresh_a) {
+        ProfScope ps(kProfSplit, 0.0, a_elems * 12.0, c.s);
+        if ((rc = split_tf32(reinterpret_cast<const float*>(g.A), pc.hi[ia], pc.lo[ia], (long long)a_elems, c.s)))
+          return rc;
+        pc.held[ia] = g.A;
+      }
+      if (fresh_b) {
+        ProfScope ps(kProfSplit, 0.0, b_elems * 12.0, c.s);
+        if ((rc = split_tf32(reinterpret_cast<const float*>(g.B), pc.hi[ib], pc.lo[ib], (long long)b_elems, c.s)))
+          return rc;
+        pc.held[ib] = g.B;
+      }
+      const Tf32Planes tp{pc.hi[ia], pc.lo[ia], pc.hi[ib], pc.lo[ib]};
+      {
+        ProfScope ps(kProfTf32, flops, bytes, c.s, prof ? gemm_tf32x3_exec_flops(g) : 0.0);
+        rc = gemm_tf32x3(g, tp, c.s);
+      }
+      for (int i = 0; i < pc.n; ++i)
+        if (pc.held[i] == g.D) pc.held[i] = nullptr;  // its source has been overwritten
+      return rc;
     }
     ProfScope ps(kProfGemmSimt, flops, bytes, c.s);
     return gemm_simt(g, c.s);
@@ -619,7 +707,17 @@ int run_batches(const std::vector<Batch>& batches, const std::vector<SrcView>& v
       if (prescale) launch_pieces(2);
       if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
       int used = 0;
+      PlaneCache planes;
+      if (L.tf32) {
+        planes.n = 3;
+        for (int i = 0; i < 3; ++i) {
+          planes.hi[i] = B.planes[i][0];
+          planes.lo[i] = B.planes[i][1];
+          planes.cap[i] = B.plane_elems[i];
+        }
+      }
       Ctx ctx{ns->compute_dtype, s, B.err, B.counters, L.n_counters, &used};
+      ctx.planes = &planes;
       int xi = 0, out_dt = pack_dt;
       if (fuse) {
         UpdateSlots& us = slots_storage();

@@ -10,18 +10,24 @@
 // (its error grows linearly with K: measured ~1.8e-6 relative at K = 256 and
 // ~9e-6 at K = 1024 when one accumulator takes the whole sum), which the Gram
 // recurrences amplify past the fp32 bar.  So every 32-deep k-block is
-// accumulated afresh in one of four TMEM buffers, and the epilogue warps fold
+// accumulated afresh in one of three TMEM buffers, and the epilogue warps fold
 // it into an fp32 register sum (round to nearest): the biased part then spans
 // only the 12 MMAs of one k-block, whatever K is.
 //
 // Layout: persistent CTA pairs on 256 x 128 output tiles (each CTA 128 rows;
 // the leader issues M=256, N=128, K=8 MMAs reading both CTAs' shared memory).
-//   - each CTA's TMA loads (24 KB of fp32 per k-block) complete on its own
-//     barrier; four converter warps in each CTA then write hi over the landed
-//     tile and lo into a second buffer of the same swizzled layout (the split
-//     is elementwise, so the layout carries over), each on its own quarter of
-//     the stage; each warp fences its writes for the tensor core and arrives
-//     on the leader's barrier, which the MMA issuer waits on;
+//   - the split is done before the product, by an HBM-bound pass that writes
+//     hi and lo as two fp32 planes of each operand (same strides as the
+//     operand; X X^T and A^2 read one pair for both operands).  The product
+//     kernel loads the four planes by TMA, each CTA's loads completing on the
+//     leader's barrier: the plain TMA -> MMA pipeline of the 16-bit kernels.
+//     Splitting in the kernel instead measured slower: in shared memory, each
+//     split needs a proxy fence before the tensor core may read it; into
+//     tensor memory (A only), the A tile becomes a third stream of loads and
+//     the converter hand-off adds latency;
+//   - the fold's per-k-block "buffer read out" arrivals use a CTA-scope
+//     release (they hand over no data): with a cluster-scope release each of
+//     them carried a memory barrier, and those paced the kernel;
 //   - MN-major B tiles use the 128-byte swizzle with 32-byte granules (the
 //     only shared-memory layout the tensor core takes for 32-bit MN-major
 //     operands), in the tensor map and in the descriptor alike;
@@ -32,6 +38,7 @@
 //     a mirror kernel then copies the strict upper triangle onto the lower one,
 //     so the result is exactly symmetric.
 // Every wait is bounded, as in the 16-bit kernels.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 
@@ -45,16 +52,14 @@ constexpr int BK32 = 32;                       // 32 x 4 B = one 128-byte swizzl
 constexpr int UMMA_K32 = 8;                    // K of one kind::tf32 MMA
 constexpr int TILE_N = 128;                    // pair tile: 256 rows x 128 columns
 constexpr int STAGES3 = 4;
-constexpr int A_OP = 128 * BK32 * 4;           // this CTA's 128 rows of A: 16 KB
-constexpr int B_OP = (TILE_N / 2) * BK32 * 4;  // this CTA's 64 columns of B: 8 KB
-constexpr int RAW_BYTES = A_OP + B_OP;         // A, B as loaded (hi written in place)
-constexpr int STAGE_BYTES3 = 2 * RAW_BYTES;    // then A lo, B lo
+constexpr int A_OP = 128 * BK32 * 4;           // this CTA's 128 rows of one A plane: 16 KB
+constexpr int B_OP = (TILE_N / 2) * BK32 * 4;  // this CTA's 64 columns of one B plane: 8 KB
+constexpr int RAW_BYTES = A_OP + B_OP;         // the hi planes of A and B; the lo planes follow
+constexpr int STAGE_BYTES3 = 2 * RAW_BYTES;
 constexpr int NUM_PBUF = 4;                    // k-block accumulators in TMEM
 constexpr int TMEM_COLS3 = NUM_PBUF * TILE_N;
-constexpr int NUM_CONV_WARPS = 4;
-constexpr int CONV_THREADS = 32 * NUM_CONV_WARPS;
-constexpr int NUM_THREADS3 = 64 + 32 * (NUM_EPI_WARPS + NUM_CONV_WARPS);
-constexpr int NUM_BARS3 = 3 * STAGES3 + 2 * NUM_PBUF + 1;
+constexpr int NUM_THREADS3 = 64 + 32 * NUM_EPI_WARPS;
+constexpr int NUM_BARS3 = 2 * STAGES3 + 2 * NUM_PBUF + 1;
 constexpr int SMEM_BYTES3 = STAGES3 * STAGE_BYTES3 + STAGING_BYTES + 1024 + 256;
 static_assert(SMEM_BYTES3 <= 232448, "exceeds the per-block shared-memory limit");
 static_assert(NUM_BARS3 * 8 + 8 <= 256, "barrier area");
@@ -73,6 +78,27 @@ __device__ __forceinline__ void mma_tf32_pair(uint32_t d_tmem, uint64_t adesc, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 64 consecutive 32-bit TMEM columns of this warp's lane quarter, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is reported on a
+// barrier of the pair (the leader's full barrier, a cluster address).
+__device__ __forceinline__ void tma_load_3d_to_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                    int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 
@@ -194,18 +220,18 @@ __device__ __forceinline__ void store_chunk_f32(const Params& p, const CUtensorM
 
 template <bool B_MN, bool SYM>
 __global__ void __launch_bounds__(NUM_THREADS3, 1)
-gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_ah, const __grid_constant__ CUtensorMap tmap_al,
+                   const __grid_constant__ CUtensorMap tmap_bh, const __grid_constant__ CUtensorMap tmap_bl,
                    const __grid_constant__ CUtensorMap tmap_d, const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + STAGES3 * STAGE_BYTES3;  // per epilogue warp: two 2 KB boxes
   uint64_t* bars = reinterpret_cast<uint64_t*>(staging + STAGING_BYTES);
-  uint64_t* full_bar = bars;                                   // [STAGES3] this CTA's loads landed
-  uint64_t* conv_bar = bars + STAGES3;                         // [STAGES3] all converter warps split the stage (leader)
-  uint64_t* empty_bar = bars + 2 * STAGES3;                    // [STAGES3] MMAs done with the stage (both CTAs)
-  uint64_t* pfull_bar = bars + 3 * STAGES3;                    // [NUM_PBUF] k-block sum ready (both CTAs)
-  uint64_t* pempty_bar = bars + 3 * STAGES3 + NUM_PBUF;        // [NUM_PBUF] k-block sum folded (leader)
-  uint64_t* drain_bar = bars + 3 * STAGES3 + 2 * NUM_PBUF;     // [1]
+  uint64_t* full_bar = bars;                                   // [STAGES3] both CTAs' loads landed (leader)
+  uint64_t* empty_bar = bars + STAGES3;                        // [STAGES3] MMAs done with the stage (both CTAs)
+  uint64_t* pfull_bar = bars + 2 * STAGES3;                    // [NUM_PBUF] k-block sum ready (both CTAs)
+  uint64_t* pempty_bar = bars + 2 * STAGES3 + NUM_PBUF;        // [NUM_PBUF] k-block sum folded (leader)
+  uint64_t* drain_bar = bars + 2 * STAGES3 + 2 * NUM_PBUF;     // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -217,7 +243,6 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES3; ++s) {
       mbar_init(smem_u32(&full_bar[s]), 1);
-      mbar_init(smem_u32(&conv_bar[s]), 2 * NUM_CONV_WARPS);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     for (int a = 0; a < NUM_PBUF; ++a) {
@@ -230,8 +255,10 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_ah)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_al)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_bh)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_bl)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_d)) : "memory");
   }
   if (warp == 1) {
@@ -246,7 +273,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int num_kb = (p.K + BK32 - 1) / BK32;
-  const uint32_t leader_conv = mapa(smem_u32(conv_bar), 0);
+  const uint32_t leader_full = mapa(smem_u32(full_bar), 0);
   const uint32_t leader_pempty = mapa(smem_u32(pempty_bar), 0);
 
   if (warp == 0) {
@@ -261,21 +288,28 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
         const int col0 = tl.TN * TILE_N + (int)rank * (TILE_N / 2);  // this CTA's columns of B
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-          const uint32_t fb = smem_u32(&full_bar[stage]);
-          mbar_expect_tx(fb, RAW_BYTES);
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES3);
+          if (leader) mbar_expect_tx(smem_u32(&full_bar[stage]), 2 * STAGE_BYTES3);
+          const uint32_t fb = leader_full + stage * 8;
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES3);  // A hi, B hi, A lo, B lo
           const uint32_t sb = sa + A_OP;
-          tma_load_3d(sa, &tmap_a, fb, kb * BK32, row0, tl.b);
-          if (B_MN) {
 #pragma unroll
-            for (int q = 0; q < TILE_N / 64; ++q)
-              tma_load_3d(sb + q * (BK32 * 128), &tmap_b, fb, col0 + q * 32, kb * BK32, tl.b);
-          } else {
-            tma_load_3d(sb, &tmap_b, fb, kb * BK32, col0, tl.b);
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t off = h * RAW_BYTES;
+            tma_load_3d_to_pair(sa + off, h ? &tmap_al : &tmap_ah, fb, kb * BK32, row0, tl.b);
+            const CUtensorMap* mb = h ? &tmap_bl : &tmap_bh;
+            if (B_MN) {
+#pragma unroll
+              for (int q = 0; q < TILE_N / 64; ++q)
+                tma_load_3d_to_pair(sb + off + q * (BK32 * 128), mb, fb, col0 + q * 32, kb * BK32, tl.b);
+            } else {
+              tma_load_3d_to_pair(sb + off, mb, fb, kb * BK32, col0, tl.b);
+            }
           }
           if (++stage == STAGES3) { stage = 0; phase ^= 1u; }
         }
       }
+      // no drain needed here: the leader's MMAs consume every issued stage,
+      // and the final cluster barrier keeps this CTA resident until then
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer (leader only)
@@ -290,7 +324,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
           const uint32_t pb = jb % NUM_PBUF;
           const uint32_t pph = (jb / NUM_PBUF) & 1u;
           if (!mbar_wait_cluster(smem_u32(&pempty_bar[pb]), pph ^ 1u, abort_flag, p.timeout_ns)) { ok = false; break; }
-          if (!mbar_wait_cluster(smem_u32(&conv_bar[stage]), phase, abort_flag, p.timeout_ns)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.timeout_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + pb * TILE_N;
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES3);
@@ -320,7 +354,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
       volatile int never = 0;
       mbar_wait(smem_u32(drain_bar), 0, &never, p.timeout_ns);
     }
-  } else if (warp < 2 + NUM_EPI_WARPS) {
+  } else {
     // ---------------------------------------------------------------- fold + epilogue (both CTAs)
     const int q = warp & 3;             // TMEM lane quarter: rows q*32 .. q*32+31 of this CTA
     const int half = (warp - 2) >> 2;   // columns half*64 .. half*64+63 of the tile
@@ -342,16 +376,15 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
         if (!w) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr = tmem_base + pb * TILE_N + (uint32_t)(half * 64) + ((uint32_t)(q * 32) << 16);
-        uint32_t r[32];
-        tmem_ld32(taddr, r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] += __uint_as_float(r[j]);
-        tmem_ld32(taddr + 32, r);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[32 + j] += __uint_as_float(r[j]);
+        uint32_t r[64];
+        tmem_ld64(taddr, r);
+        // the buffer is free once read out: release it before folding, which
+        // keeps the fold's adds off the MMA issuer's path
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) remote_arrive(leader_pempty + pb * 8);
+        if (lane == 0) remote_arrive_cta(leader_pempty + pb * 8);  // no data handed over
+#pragma unroll
+        for (int j = 0; j < 64; ++j) acc[j] += __uint_as_float(r[j]);
       }
       if (!ok) break;
       const float f = matrix_scale(p.scale, p.scale_pow, tl.b);
@@ -366,36 +399,6 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_cons
     }
     if (lane == 0) bulk_wait_all0();  // this warp's output stores have completed
     __syncwarp();
-  } else {
-    // ---------------------------------------------------------------- converters (both CTAs)
-    // Each converter warp splits its own quarter of every stage and signals
-    // the leader itself, so the warps pipeline across stages: no named
-    // barrier, one arrival per warp and CTA on the leader's barrier.
-    const int cw = warp - (2 + NUM_EPI_WARPS);
-    int stage = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int t = pair; t < p.total_tiles && ok; t += npairs) {
-      for (int kb = 0; kb < num_kb; ++kb) {
-        // every lane waits itself (acquiring the landed bytes); the vote keeps
-        // the warp together if the wait runs out for some lanes only
-        const bool got = mbar_wait(smem_u32(&full_bar[stage]), phase, abort_flag, p.timeout_ns);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        float4* raw = reinterpret_cast<float4*>(smem + stage * STAGE_BYTES3);
-        float4* lo = raw + RAW_BYTES / 16;
-#pragma unroll 4
-        for (int i = cw * 32 + lane; i < RAW_BYTES / 16; i += CONV_THREADS) {
-          const float4 x = raw[i];
-          const float4 h = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
-          raw[i] = h;
-          lo[i] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
-        }
-        fence_async_smem();  // the tensor core reads what these lanes wrote
-        __syncwarp();
-        if (lane == 0) remote_arrive(leader_conv + stage * 8);
-        if (++stage == STAGES3) { stage = 0; phase ^= 1u; }
-      }
-    }
   }
 
   __syncwarp();
@@ -438,9 +441,19 @@ __global__ void __launch_bounds__(256) mirror_upper_kernel(float* D, int n, int 
   }
 }
 
+// hi = src rounded to TF32, lo = src - hi (exact in fp32), over n4 float4s.
+__global__ void __launch_bounds__(256) split_tf32_kernel(const float4* __restrict__ src, float4* __restrict__ hi,
+                                                         float4* __restrict__ lo, long long n4) {
+  for (long long i = blockIdx.x * 256LL + threadIdx.x; i < n4; i += (long long)gridDim.x * 256) {
+    const float4 x = src[i];
+    const float4 h = make_float4(tf32_hi(x.x), tf32_hi(x.y), tf32_hi(x.z), tf32_hi(x.w));
+    hi[i] = h;
+    lo[i] = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+  }
+}
+
 template <bool B_MN, bool SYM>
-static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& md, const Params& p,
-                  cudaStream_t s) {
+static int launch(const CUtensorMap (&m)[5], const Params& p, cudaStream_t s) {
   static std::atomic<int> max_pairs_of[kMaxDevices];
   const int dev = current_device();
   if (dev < 0) return (int)cudaErrorInvalidDevice;
@@ -469,7 +482,7 @@ static int launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMa
   }
   const int pairs = p.total_tiles < max_pairs ? p.total_tiles : max_pairs;
   cfg.gridDim = dim3(2 * pairs);
-  return (int)cudaLaunchKernelEx(&cfg, kern, ma, mb, md, p);
+  return (int)cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], p);
 }
 
 }  // namespace tf32k
@@ -485,7 +498,21 @@ double gemm_tf32x3_exec_flops(const GemmDesc& g) {
   return 3.0 * 2.0 * tiles * 256.0 * TILE_N * k_pad * g.batch;  // hi*hi + hi*lo + lo*hi
 }
 
-int gemm_tf32x3(const GemmDesc& g, cudaStream_t s) {
+int split_tf32(const float* src, float* hi, float* lo, long long elems, cudaStream_t s) {
+  using namespace tc::tf32k;
+  if (elems <= 0) return 0;
+  if ((elems & 3) || (reinterpret_cast<uintptr_t>(src) & 15) || (reinterpret_cast<uintptr_t>(hi) & 15) ||
+      (reinterpret_cast<uintptr_t>(lo) & 15))
+    return (int)cudaErrorInvalidValue;
+  const long long n4 = elems / 4;
+  const long long want = (n4 + 255) / 256;
+  const int blocks = (int)std::min<long long>(want, 8LL * num_sms());
+  split_tf32_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(src), reinterpret_cast<float4*>(hi),
+                                           reinterpret_cast<float4*>(lo), n4);
+  return (int)cudaGetLastError();
+}
+
+int gemm_tf32x3(const GemmDesc& g, const Tf32Planes& pl, cudaStream_t s) {
   using namespace tc;
   using namespace tc::tf32k;
   if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return 0;
@@ -513,19 +540,26 @@ int gemm_tf32x3(const GemmDesc& g, cudaStream_t s) {
   p.err = g.err;
   p.timeout_ns = wait_timeout_ns();
 
-  CUtensorMap ma, mb, md;
-  if (!encode_map(&ma, kFP32, g.A, g.K, g.M, g.batch, g.lda, g.a_bs, BK32, 128)) return (int)cudaErrorInvalidValue;
+  // m: A hi, A lo, B hi, B lo (planes with the operands' strides), D
+  CUtensorMap m[5];
+  if (!pl.a_hi || !pl.a_lo || !pl.b_hi || !pl.b_lo) return (int)cudaErrorInvalidValue;
+  const float* ap[2] = {pl.a_hi, pl.a_lo};
+  const float* bp[2] = {pl.b_hi, pl.b_lo};
   const bool bmn = !g.b_kmajor;
-  if (bmn) {
-    if (!encode_map(&mb, kFP32, g.B, g.N, g.K, g.batch, g.ldb, g.b_bs, 32, BK32, kTmaSw128Atom32))
-      return (int)cudaErrorInvalidValue;
-  } else {
-    if (!encode_map(&mb, kFP32, g.B, g.K, g.N, g.batch, g.ldb, g.b_bs, BK32, TILE_N / 2)) return (int)cudaErrorInvalidValue;
+  for (int h = 0; h < 2; ++h) {
+    if (!encode_map(&m[h], kFP32, ap[h], g.K, g.M, g.batch, g.lda, g.a_bs, BK32, 128)) return (int)cudaErrorInvalidValue;
+    if (bmn) {
+      if (!encode_map(&m[2 + h], kFP32, bp[h], g.N, g.K, g.batch, g.ldb, g.b_bs, 32, BK32, kTmaSw128Atom32))
+        return (int)cudaErrorInvalidValue;
+    } else {
+      if (!encode_map(&m[2 + h], kFP32, bp[h], g.K, g.N, g.batch, g.ldb, g.b_bs, BK32, TILE_N / 2))
+        return (int)cudaErrorInvalidValue;
+    }
   }
-  if (!encode_map(&md, kFP32, g.D, g.N, g.M, g.batch, g.ldd, g.d_bs, 16, 32, kTmaSw64)) return (int)cudaErrorInvalidValue;
+  if (!encode_map(&m[4], kFP32, g.D, g.N, g.M, g.batch, g.ldd, g.d_bs, 16, 32, kTmaSw64)) return (int)cudaErrorInvalidValue;
   int rc;
-  if (g.symmetric) rc = bmn ? launch<true, true>(ma, mb, md, p, s) : launch<false, true>(ma, mb, md, p, s);
-  else rc = bmn ? launch<true, false>(ma, mb, md, p, s) : launch<false, false>(ma, mb, md, p, s);
+  if (g.symmetric) rc = bmn ? launch<true, true>(m, p, s) : launch<false, true>(m, p, s);
+  else rc = bmn ? launch<true, false>(m, p, s) : launch<false, false>(m, p, s);
   if (rc != 0 || !g.symmetric) return rc;
   const int T = (g.M + 31) / 32;
   const int ntri = T * (T + 1) / 2;

@@ -116,8 +116,17 @@ constexpr int kChainMaxProducts = 24;
 // three MMAs per product term.  The algorithmic count is 2 M N K per matrix.
 double gemm_tc_exec_flops(const GemmDesc& g);
 double gemm_tf32x3_exec_flops(const GemmDesc& g);
-// Tensor-core path for fp32 operands (3xTF32, paired CTAs): fp32 A, B, C and D.
-int gemm_tf32x3(const GemmDesc& g, cudaStream_t s);
+// Tensor-core path for fp32 operands (3xTF32, paired CTAs): fp32 C and D; A
+// and B are read as their TF32 splits, hi = x rounded to TF32 and lo = x - hi,
+// stored as fp32 planes with the operand's own strides (split_tf32 writes
+// them).  g.A / g.B are not read.
+struct Tf32Planes {
+  const float* a_hi; const float* a_lo;
+  const float* b_hi; const float* b_lo;
+};
+int gemm_tf32x3(const GemmDesc& g, const Tf32Planes& planes, cudaStream_t s);
+// hi / lo planes of `elems` fp32 values (a multiple of 4, 16-byte aligned).
+int split_tf32(const float* src, float* hi, float* lo, long long elems, cudaStream_t s);
 // SIMT path (any dtype, fp32 math): fp32 products with fewer than 256 rows.
 int gemm_simt(const GemmDesc& g, cudaStream_t s);
 

@@ -530,6 +530,14 @@ __device__ __forceinline__ void commit_pair(uint32_t bar, uint16_t mask) {
 __device__ __forceinline__ void remote_arrive(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
+// Arrive on a barrier of a CTA of the cluster with release at CTA scope only:
+// for signals that hand over no memory contents, such as "this TMEM buffer
+// has been read out" (after tcgen05.wait::ld and a tcgen05 fence), where the
+// cluster-scope release of remote_arrive would add a memory barrier to every
+// arrival.
+__device__ __forceinline__ void remote_arrive_cta(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
 // Store to the same shared-memory object in another CTA of the cluster (address from mapa).
 __device__ __forceinline__ void st_cluster_s32(uint32_t addr_cluster, int v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr_cluster), "r"(v) : "memory");
