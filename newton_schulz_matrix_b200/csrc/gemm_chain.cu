@@ -370,7 +370,7 @@ gemm_chain_kernel(const __grid_constant__ ChainParams cp,
           __syncwarp();
           if (lane == 0) {
             if (leader) mbar_arrive(smem_u32(&tempty_bar[acc]));
-            else remote_arrive(leader_tempty + acc * 8);
+            else remote_arrive_cta(leader_tempty + acc * 8);  // accumulator read out: no data handed over
           }
         }
         if constexpr (UPD) {

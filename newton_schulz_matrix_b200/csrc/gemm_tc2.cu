@@ -310,7 +310,7 @@ gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_consta
           __syncwarp();
           if (lane == 0) {
             if (leader) mbar_arrive(smem_u32(&tempty_bar[acc]));
-            else remote_arrive(leader_tempty + acc * 8);
+            else remote_arrive_cta(leader_tempty + acc * 8);  // accumulator read out: no data handed over
           }
         }
         if constexpr (UPD) {

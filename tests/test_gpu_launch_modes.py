@@ -123,3 +123,21 @@ def test_profile_of_a_default_step():
     assert prof["tc_product"]["launches"] == 5 and prof["tc_product[symmetric]"]["launches"] == 10
     flops = prof["tc_product"]["flops"] + prof["tc_product[symmetric]"]["flops"]
     assert flops == pytest.approx(nsm.muon_ns_flops(512, 1024), rel=1e-12)
+
+
+def test_fp32_operand_splits_are_reused():
+    """An fp32 chain with n >= 256 reads its operands as TF32 hi/lo planes
+    written by split_tf32_kernel, once per buffer content: per standard
+    iteration X (reused by the update product X <- aX + BX), A and B, at
+    12 bytes per element (x read, hi and lo written)."""
+    n, m, count, iters = 512, 1024, 2, 5
+    X = [synth.gaussian(n, m, 40 + i, "cuda") for i in range(count)]
+    nsm.muon_profile_begin()
+    nsm.muon_ns_batched(X, compute_dtype="fp32")
+    prof = {r["kernel"]: r for r in nsm.muon_profile_end()}
+    assert prof["tc_product[3xtf32]"]["launches"] == 3 * iters
+    split = prof["split_tf32_kernel"]
+    assert split["launches"] == 3 * iters
+    elems_per_iter = count * (n * m + 2 * n * n)
+    assert split["bytes"] == pytest.approx(12.0 * elems_per_iter * iters, rel=1e-12)
+    assert all(torch.isfinite(x).all() for x in X)
