@@ -54,8 +54,8 @@ KERNEL_SOURCES = {
 # launch list of `python bench.py --workload <w> --compute <c> --steps 1
 # --warmup 1` with --metrics dram__bytes_read.sum,dram__bytes_write.sum).
 MEASURED_TRAFFIC: dict = {
-    ("kimi-k2", "fp16", "tc_product"): ("c25d1a976625a897", 17.73e9),
-    ("kimi-k2", "fp16", "tc_product[symmetric]"): ("c25d1a976625a897", 6.96e9),
+    ("kimi-k2", "fp16", "tc_product"): ("96748409045dea26", 17.41e9),
+    ("kimi-k2", "fp16", "tc_product[symmetric]"): ("96748409045dea26", 7.03e9),
     # captured on the 16-matrix dense16 set (0.673 GB per launch), x 4 for the
     # 64-matrix dense set: the products' traffic grows with the matrix count
     ("dense", "fp32", "tc_product[3xtf32]"): ("9a6231d04d71d8ae", 2.69e9),
