@@ -257,9 +257,10 @@ int plane_pair(PlaneCache& pc, const void* src, size_t elems, int avoid, bool* f
   int best = -1;
   for (int i = 0; i < pc.n; ++i) {
     if (i == avoid || pc.cap[i] < elems) continue;
-    // an empty pair first, then the smallest that fits
-    if (best < 0 || (pc.held[i] == nullptr && pc.held[best] != nullptr) ||
-        ((pc.held[i] == nullptr) == (pc.held[best] == nullptr) && pc.cap[i] < pc.cap[best]))
+    // the smallest pair that fits (an n x n operand never takes the X-sized
+    // pair that the update product's X needs), an empty one among equals
+    if (best < 0 || pc.cap[i] < pc.cap[best] ||
+        (pc.cap[i] == pc.cap[best] && pc.held[i] == nullptr && pc.held[best] != nullptr))
       best = i;
   }
   *fresh = true;
