@@ -211,6 +211,26 @@ __device__ __forceinline__ uint16_t to_bits(float v, int dt) {
 __device__ __forceinline__ uint32_t sw64(int row, int chunk16) {
   return (uint32_t)(row * 64 + ((chunk16 ^ ((row >> 1) & 3)) << 4));
 }
+// T = S^T for a warp's 32 x 32 box of 16-bit values, both in the sw64 layout.
+// Round g moves column block g of the four 8 x 8 row blocks of S: ldmatrix
+// .trans reads them (lane l addresses row l of S) transposed into the
+// fragment layout, and stmatrix writes each as row block g of T (lane l
+// addresses row 8 g + l % 8 of block l / 8): 8 instructions per lane.
+__device__ __forceinline__ void transpose_box16(const uint8_t* S, uint8_t* T, int lane) {
+  const uint32_t s0 = smem_u32(S), t0 = smem_u32(T);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t r0, r1, r2, r3;
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(s0 + sw64(lane, g))
+                 : "memory");
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(
+                     t0 + sw64(g * 8 + (lane & 7), lane >> 3)),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+  }
+}
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
@@ -310,11 +330,14 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMa
   // the staging boxes are free once the previous chunk's stores have read them
   if (lane == 0) bulk_wait_read0();
   __syncwarp();
-  if (SYM && (mirror || diag_box)) {
-    // transposed box: T[j][lane] = v[j]
+  uint4 dq[4];
+  pack_row32(v, p.d_dtype, dq);
 #pragma unroll
-    for (int j = 0; j < 32; ++j)
-      *reinterpret_cast<uint16_t*>(T + sw64(j, lane >> 3) + (lane & 7) * 2) = to_bits(v[j], p.d_dtype);
+  for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(S + sw64(lane, k)) = dq[k];
+  if (SYM && (mirror || diag_box)) {
+    // transposed box T = S^T
+    __syncwarp();
+    transpose_box16(S, T, lane);
     if (diag_box) {
       __syncwarp();
       // below the diagonal take the transposed value, so the box is exactly symmetric
@@ -322,8 +345,6 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMa
 #pragma unroll
       for (int k = 0; k < 4; ++k) tq[k] = *reinterpret_cast<const uint4*>(T + sw64(lane, k));
       const uint16_t* te = reinterpret_cast<const uint16_t*>(tq);
-      uint4 dq[4];
-      pack_row32(v, p.d_dtype, dq);
       uint16_t* de = reinterpret_cast<uint16_t*>(dq);
 #pragma unroll
       for (int j = 0; j < 32; ++j)
@@ -331,12 +352,6 @@ __device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMa
 #pragma unroll
       for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(S + sw64(lane, k)) = dq[k];
     }
-  }
-  if (!diag_box) {
-    uint4 dq[4];
-    pack_row32(v, p.d_dtype, dq);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(S + sw64(lane, k)) = dq[k];
   }
   fence_async_smem();
   __syncwarp();
