@@ -175,9 +175,16 @@ __device__ __forceinline__ Tile32 decode_t32(const Params& p, int t) {
 __device__ __forceinline__ void store_chunk_f32(const Params& p, const CUtensorMap* tmap_d, int b, int gi_base,
                                                 int gj0, int lane, const float* s, float f, uint8_t* S, uint8_t* T) {
   const int gi = gi_base + lane;
+  // multiplications by 1 and a zero identity term are skipped (warp-uniform
+  // tests); the identity's diagonal lies in the boxes with gj0 == gi_base only
   float v[32];
+  if (p.c_acc != 1.f) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = p.c_acc * s[j];
+    for (int j = 0; j < 32; ++j) v[j] = p.c_acc * s[j];
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = s[j];
+  }
   if (p.C != nullptr && gi < p.M) {
     const float* crow = reinterpret_cast<const float*>(p.C) + (long long)b * p.c_bs + (long long)gi * p.ldc + gj0;
     if (gj0 + 32 <= p.N) {
@@ -196,10 +203,14 @@ __device__ __forceinline__ void store_chunk_f32(const Params& p, const CUtensorM
         if (gj0 + j < p.N) v[j] += p.c_in * crow[j];
     }
   }
+  if (f != 1.f) {
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    v[j] *= f;
-    if (gj0 + j == gi) v[j] += p.c_eye;
+    for (int j = 0; j < 32; ++j) v[j] *= f;
+  }
+  if (p.c_eye != 0.f && gj0 == gi_base) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j == lane) v[j] += p.c_eye;
   }
   if (lane == 0) bulk_wait_read0();  // the boxes are free once earlier stores have read them
   __syncwarp();
