@@ -54,12 +54,12 @@ KERNEL_SOURCES = {
 # launch list of `python bench.py --workload <w> --compute <c> --steps 1
 # --warmup 1` with --metrics dram__bytes_read.sum,dram__bytes_write.sum).
 MEASURED_TRAFFIC: dict = {
-    ("kimi-k2", "fp16", "tc_product"): ("d80c824df03c426f", 17.47e9),
-    ("kimi-k2", "fp16", "tc_product[symmetric]"): ("d80c824df03c426f", 7.03e9),
+    ("kimi-k2", "fp16", "tc_product"): ("b6ba3e11bb008431", 17.47e9),
+    ("kimi-k2", "fp16", "tc_product[symmetric]"): ("b6ba3e11bb008431", 7.03e9),
     # captured on the 16-matrix dense16 set (0.674 GB per launch), x 4 for the
     # 64-matrix dense set: the products' traffic grows with the matrix count
-    ("dense", "fp32", "tc_product[3xtf32]"): ("2fd230dbda414673", 2.69e9),
-    ("dense16", "fp32", "tc_product[3xtf32]"): ("2fd230dbda414673", 0.674e9),
+    ("dense", "fp32", "tc_product[3xtf32]"): ("59e49be3ff193377", 2.69e9),
+    ("dense16", "fp32", "tc_product[3xtf32]"): ("59e49be3ff193377", 0.674e9),
 }
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)

@@ -254,14 +254,6 @@ __device__ __forceinline__ void pack_row32(const float* v, int dt, uint4 (&q)[4]
   }
 }
 
-// One 32 x 32 chunk of the output: this warp's 32 tile rows (one per lane,
-// TMEM lane quarter q) times columns [gj0, gj0 + 32).  `creg` holds the C row
-// segment when `c_ready` (loaded before the TMEM read to hide its latency).
-// Symmetric products: off-diagonal 128-blocks are stored directly and
-// transposed; inside a diagonal 128-block, boxes above the diagonal are stored
-// both ways, boxes below are skipped (their transposes cover them) and the box
-// on the diagonal is made exactly symmetric in shared memory first.
-// S and T are this warp's two staging boxes (1024-byte aligned).
 // v = f (c_acc acc + c_in C) + c_eye I for one 32-column chunk of row gi;
 // the C term is added by the caller.  Multiplications by 1 and a zero
 // identity term are skipped (warp-uniform tests): the default chains have
@@ -288,6 +280,14 @@ __device__ __forceinline__ void finish32(const Params& p, float f, int gi_base, 
   }
 }
 
+// One 32 x 32 chunk of the output: this warp's 32 tile rows (one per lane,
+// TMEM lane quarter q) times columns [gj0, gj0 + 32).  `creg` holds the C row
+// segment when `c_ready` (loaded before the TMEM read to hide its latency).
+// Symmetric products: off-diagonal 128-blocks are stored directly and
+// transposed; inside a diagonal 128-block, boxes above the diagonal are stored
+// both ways, boxes below are skipped (their transposes cover them) and the box
+// on the diagonal is made exactly symmetric in shared memory first.
+// S and T are this warp's two staging boxes (1024-byte aligned).
 template <bool SYM>
 __device__ __forceinline__ void epilogue_chunk(const Params& p, const CUtensorMap* tmap_d, const Tile& t, int q,
                                                int lane, int chunk, const uint32_t (&acc)[32],
