@@ -82,6 +82,25 @@ def test_ns_workspace_size(lib):
     assert lib.muon_ns_workspace_size(1, 64, 64, ctypes.byref(bad)) == 0
 
 
+def test_fp32_workspace_holds_the_tf32_planes(lib):
+    """fp32 chains whose products run as 3xTF32 (n >= 256) also hold their
+    operands' TF32 hi / lo planes, one X-sized and two n x n pairs:
+    2 (n m + 2 n^2) x 4 bytes per matrix on top of the chain's own buffers
+    (twice the 16-bit ones); the fused small-matrix path (n < 256) holds none."""
+    ns16, _a = _ns()
+    ns32, _b = _ns(compute="fp32")
+
+    def per_matrix(ns, n, m):
+        return lib.muon_ns_workspace_size(2, n, m, ctypes.byref(ns)) - lib.muon_ns_workspace_size(1, n, m, ctypes.byref(ns))
+
+    n, m = 512, 1024
+    planes = 2 * (n * m + 2 * n * n) * 4
+    extra = per_matrix(ns32, n, m) - 2 * per_matrix(ns16, n, m)
+    assert planes - 4096 < extra <= planes  # less the doubled per-matrix partials and counters
+    n, m = 128, 256
+    assert abs(per_matrix(ns32, n, m) - 2 * per_matrix(ns16, n, m)) < 4096
+
+
 def _fake_group(rows, cols, count, wdt=nsm.BF16, gdt=nsm.BF16, ptr=1 << 20):
     arrs = [(ctypes.c_void_p * count)(*[ptr + 4096 * i for i in range(count)]) for _ in range(3)]
     return nsm._Group(rows, cols, count, wdt, gdt, *arrs), arrs
